@@ -1,0 +1,141 @@
+"""CPU oracle of the group-32 symmetric INT4 quantizer path.
+
+TEST INFRASTRUCTURE: only the tests, the smoke check and the benchmark's CPU
+baseline use it.  The product package never imports it.  The arithmetic lives
+in ``qat4_oracle.c`` (plain C, fp64 sums); this module only marshals NumPy
+arrays into it.  ``twin.py`` is a second, independent NumPy implementation for
+tiny inputs.
+"""
+from __future__ import annotations
+
+import ctypes as ct
+
+import numpy as np
+
+from .build import build as _build
+
+_LIB = None
+_P = ct.c_void_p
+_I64 = ct.c_int64
+
+
+def lib():
+    global _LIB
+    if _LIB is None:
+        _LIB = ct.CDLL(_build())
+        L = _LIB
+        L.oracle_set_threads.argtypes = [ct.c_int]
+        L.oracle_set_threads.restype = ct.c_int
+        L.oracle_hessian.argtypes = [_P, _I64, _I64, _P]
+        L.oracle_hessian_entries.argtypes = [_P, _I64, _I64, _P, _P, _I64, _P]
+        L.oracle_hessian_block.argtypes = [_P, _I64, _I64, _I64, _I64, _I64, _I64, _P]
+        L.oracle_scale_search.argtypes = [_P, _I64, _I64, _P, _I64, _P, ct.c_int32, _P, _P, _P, _P]
+        L.oracle_lsq_fwd.argtypes = [_P, _P, _I64, _I64, _P]
+        L.oracle_lsq_bwd.argtypes = [_P, _P, _P, ct.c_int, _I64, _I64, ct.c_float, _P, _P]
+        L.oracle_pack_w4a16.argtypes = [_P, _P, _I64, _I64, _P, _P]
+        L.oracle_codes.argtypes = [_P, _P, _I64, _I64, _P]
+        for f in ("oracle_hessian", "oracle_hessian_entries", "oracle_hessian_block",
+                  "oracle_scale_search", "oracle_lsq_fwd", "oracle_lsq_bwd",
+                  "oracle_pack_w4a16", "oracle_codes"):
+            getattr(L, f).restype = None
+    return _LIB
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(_P)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def set_threads(n: int = 0) -> int:
+    """Set the OpenMP thread count (n <= 0 keeps it); returns the count in use."""
+    return lib().oracle_set_threads(int(n))
+
+
+def hessian(X_bits: np.ndarray) -> np.ndarray:
+    """H = X^T X / n in float64 for X given as bf16 bits [n, C]."""
+    X = _c(X_bits, np.uint16)
+    n, C = X.shape
+    H = np.empty((C, C), np.float64)
+    lib().oracle_hessian(_p(X), n, C, _p(H))
+    return H
+
+
+def hessian_entries(X_bits: np.ndarray, ii, jj) -> np.ndarray:
+    X = _c(X_bits, np.uint16)
+    n, C = X.shape
+    ii = _c(ii, np.int64)
+    jj = _c(jj, np.int64)
+    out = np.empty(ii.size, np.float64)
+    lib().oracle_hessian_entries(_p(X), n, C, _p(ii), _p(jj), ii.size, _p(out))
+    return out
+
+
+def hessian_block(X_bits: np.ndarray, r0: int, nr: int, c0: int, nc: int) -> np.ndarray:
+    X = _c(X_bits, np.uint16)
+    n, C = X.shape
+    out = np.empty((nr, nc), np.float64)
+    lib().oracle_hessian_block(_p(X), n, C, r0, nr, c0, nc, _p(out))
+    return out
+
+
+def scale_search(W: np.ndarray, H: np.ndarray, alpha: np.ndarray, *, all_err: bool = False):
+    """Returns (delta f32 [R,G], idx i32 [R,G], best_err f64 [R,G][, all f64 [R,G,K]])."""
+    W = _c(W, np.float32)
+    H = _c(H, np.float32)
+    alpha = _c(alpha, np.float32)
+    R, C = W.shape
+    G = C // 32
+    K = alpha.size
+    delta = np.empty((R, G), np.float32)
+    idx = np.empty((R, G), np.int32)
+    best = np.empty((R, G), np.float64)
+    allv = np.empty((R, G, K), np.float64) if all_err else None
+    lib().oracle_scale_search(_p(W), R, C, _p(H), H.shape[1], _p(alpha), K, _p(delta), _p(idx),
+                              _p(best), _p(allv) if all_err else None)
+    return (delta, idx, best, allv) if all_err else (delta, idx, best)
+
+
+def lsq_fwd(W: np.ndarray, delta: np.ndarray) -> np.ndarray:
+    W = _c(W, np.float32)
+    delta = _c(delta, np.float32)
+    R, C = W.shape
+    Q = np.empty_like(W)
+    lib().oracle_lsq_fwd(_p(W), _p(delta), R, C, _p(Q))
+    return Q
+
+
+def lsq_bwd(W: np.ndarray, delta: np.ndarray, G: np.ndarray, grad_scale: float):
+    """G: float32 array, or uint16 bf16 bits.  Returns (grad_W f32, grad_delta f64)."""
+    W = _c(W, np.float32)
+    delta = _c(delta, np.float32)
+    is_bf16 = np.asarray(G).dtype == np.uint16
+    G = _c(G, np.uint16 if is_bf16 else np.float32)
+    R, C = W.shape
+    gW = np.empty_like(W)
+    gD = np.empty((R, C // 32), np.float64)
+    lib().oracle_lsq_bwd(_p(W), _p(delta), _p(G), int(is_bf16), R, C, ct.c_float(grad_scale),
+                         _p(gW), _p(gD))
+    return gW, gD
+
+
+def pack_w4a16(W: np.ndarray, delta: np.ndarray):
+    """Returns (packed uint8 [R, C/2], scale16 bits uint16 [R, C/32])."""
+    W = _c(W, np.float32)
+    delta = _c(delta, np.float32)
+    R, C = W.shape
+    packed = np.empty((R, C // 2), np.uint8)
+    s16 = np.empty((R, C // 32), np.uint16)
+    lib().oracle_pack_w4a16(_p(W), _p(delta), R, C, _p(packed), _p(s16))
+    return packed, s16
+
+
+def codes(W: np.ndarray, delta: np.ndarray) -> np.ndarray:
+    W = _c(W, np.float32)
+    delta = _c(delta, np.float32)
+    R, C = W.shape
+    out = np.empty((R, C), np.int8)
+    lib().oracle_codes(_p(W), _p(delta), R, C, _p(out))
+    return out

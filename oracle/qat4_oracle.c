@@ -1,0 +1,309 @@
+/*
+ * qat4_oracle.c -- plain CPU reference of the group-32 symmetric INT4 weight
+ * quantizer (calibration Hessian, Hessian-weighted scale search, LSQ forward /
+ * backward, W4A16 packing).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, loads or
+ * calls this file; only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg do.  It shares no code, header, table or helper with the
+ * CUDA kernels.
+ *
+ * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fopenmp -fPIC
+ *        -shared  (x86-64 SSE arithmetic: every float operation below is one
+ *        IEEE binary32 operation in round-to-nearest-even, every double
+ *        operation one binary64 operation; no contraction into FMA).
+ *
+ * Sources (web pages on the method):
+ *  [card]  model card "Opt.Gear-1B-qat-int4-per-channel-unquantized",
+ *          section "Quantization Configuration" (symmetric, zero-point 0;
+ *          the per-group objective  Delta* = argmin ||W X - Q_Delta(W) X||_F^2)
+ *          and "QAT Highlights" (group size 32, same grid at init/QAT/export).
+ *  [blog]  "Opt.Gear-QAT: Preserving On-Device Performance with QAT",
+ *          section "Quantization parameters of Opt.Gear-1B" (group size 32,
+ *          symmetric), section 1 "Quantization scale is important" (uniform
+ *          projection onto a limited integer grid with step Delta), section 2
+ *          "Hessian-based scale initialize" (layer sensitivity from
+ *          calibration inputs, second-order output reconstruction), section 3
+ *          "LSQ-based QAT" (forward emulates the deployment INT4 grid; STE for
+ *          round; step-size gradient normalised by the group's element count
+ *          and the number of positive levels).
+ *  The printed formulas of [blog] sections 1-3 were lost; where a step is not
+ *  fixed by the surviving text the plainest reading is taken:
+ *    Q_Delta(w) = Delta * clamp(rint(w / Delta), -8, 7), rint = half-to-even;
+ *    H = X^T X / n;  Delta_k = alpha_k * (max|w_g| / 7);
+ *    objective per group = e H_gg e^T with e = w_g - Q(w_g) (block-diagonal
+ *    reading of the objective, other groups held at zero error);
+ *    LSQ (Esser et al., "Learned Step Size Quantization", ICLR 2020) step
+ *    gradient with scale s = 1/sqrt(32 * 7).
+ *
+ * Pins: none of these functions can be pinned to a number printed on the
+ * pages (they print no worked example of the quantizer).  Each is pinned by
+ * mathematics instead -- closed forms, invariants, special cases and brute
+ * force on tiny inputs -- in the CPU test-suite.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define GROUP 32
+#define QMIN (-8.0f)
+#define QMAX (7.0f)
+
+/* ---------------------------------------------------------------- helpers */
+
+int oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
+
+/* bf16 bit pattern -> float: the 16 bits are the top half of a binary32. */
+static float bf16_to_float(uint16_t bits)
+{
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* v = w / Delta as one IEEE binary32 division ([blog] section 1).
+ * Delta == 0 only happens for an all-zero group; v is then taken as 0. */
+static float scaled(float w, float delta)
+{
+    if (delta == 0.0f) return 0.0f;
+    return w / delta;
+}
+
+/* q = clamp(round(v), -8, 7), round = round-half-to-even ([card]
+ * "Symmetric (zero-point fixed at 0)"; INT4 two's-complement range). */
+static float code_of(float v)
+{
+    float q = rintf(v);
+    if (q < QMIN) q = QMIN;
+    if (q > QMAX) q = QMAX;
+    return q;
+}
+
+/* Q_Delta(w) = Delta * q, one binary32 multiply. */
+static float fake_quant(float w, float delta)
+{
+    float q = code_of(scaled(w, delta));
+    return delta * q;
+}
+
+/* ----------------------------------------------------- (a) Hessian H=X^TX/n
+ * [blog] section 2: layer sensitivity estimated from calibration inputs; the
+ * second-order output-reconstruction Hessian of ||W X - Q X||^2 is X^T X
+ * (up to the 1/n normalisation).  Products of bf16 values are exact in
+ * double; the sum over the n calibration rows is taken in double.
+ * X: bf16 bits, row-major [n, C].  H: double, row-major [C, C] (full). */
+void oracle_hessian(const uint16_t *X, int64_t n, int64_t C, double *H)
+{
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t i = 0; i < C; ++i) {
+        for (int64_t j = 0; j < C; ++j) {
+            double s = 0.0;
+            for (int64_t t = 0; t < n; ++t) {
+                double xi = (double)bf16_to_float(X[t * C + i]);
+                double xj = (double)bf16_to_float(X[t * C + j]);
+                s += xi * xj;
+            }
+            H[i * C + j] = s / (double)n;
+        }
+    }
+}
+
+/* Selected entries H[ii[m], jj[m]] only (for sampled checks of large X). */
+void oracle_hessian_entries(const uint16_t *X, int64_t n, int64_t C,
+                            const int64_t *ii, const int64_t *jj, int64_t count,
+                            double *out)
+{
+    #pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t m = 0; m < count; ++m) {
+        int64_t i = ii[m], j = jj[m];
+        double s = 0.0;
+        for (int64_t t = 0; t < n; ++t) {
+            double xi = (double)bf16_to_float(X[t * C + i]);
+            double xj = (double)bf16_to_float(X[t * C + j]);
+            s += xi * xj;
+        }
+        out[m] = s / (double)n;
+    }
+}
+
+/* A dense block H[r0:r0+nr, c0:c0+nc] (row-major [nr, nc] in out). */
+void oracle_hessian_block(const uint16_t *X, int64_t n, int64_t C,
+                          int64_t r0, int64_t nr, int64_t c0, int64_t nc, double *out)
+{
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t a = 0; a < nr; ++a) {
+        for (int64_t b = 0; b < nc; ++b) {
+            double s = 0.0;
+            for (int64_t t = 0; t < n; ++t) {
+                double xi = (double)bf16_to_float(X[t * C + r0 + a]);
+                double xj = (double)bf16_to_float(X[t * C + c0 + b]);
+                s += xi * xj;
+            }
+            out[a * nc + b] = s / (double)n;
+        }
+    }
+}
+
+/* ------------------------------------------ (b) Hessian-weighted scale search
+ * [card] "Quantization Configuration": for each quantization group the scale
+ * is initialised as Delta* = argmin_Delta ||W X - Q_Delta(W) X||_F^2, searched
+ * here over the finite grid Delta_k = alpha_k * (max|w_g| / 7).  For one
+ * group g of row r the objective is the quadratic form e H_gg e^T with
+ * e = w_g - Q_{Delta_k}(w_g) (computed as binary32 values, as the quantized
+ * weights are stored) and H_gg the 32x32 diagonal block of H.  Every
+ * candidate is evaluated; the smallest index reaching the minimum wins.
+ *
+ * W: float [R, C] row-major; H: float, row stride ldh (only the diagonal
+ * 32x32 blocks are read); alpha: float [K].
+ * Outputs per (r, g), row-major [R, C/32]: delta (float), idx (int32),
+ * best_err (double).  all_err (nullable): double [R, C/32, K]. */
+void oracle_scale_search(const float *W, int64_t R, int64_t C,
+                         const float *H, int64_t ldh,
+                         const float *alpha, int32_t K,
+                         float *delta_out, int32_t *idx_out, double *best_err,
+                         double *all_err)
+{
+    const int64_t G = C / GROUP;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t g = 0; g < G; ++g) {
+            const float *w = W + r * C + g * GROUP;
+            const float *Hg = H + (g * GROUP) * ldh + g * GROUP;
+            float m = 0.0f;
+            for (int i = 0; i < GROUP; ++i) {
+                float a = fabsf(w[i]);
+                if (a > m) m = a;
+            }
+            float base = m / 7.0f;
+            int32_t best_k = -1;
+            double best = 0.0;
+            float best_delta = 0.0f;
+            for (int32_t k = 0; k < K; ++k) {
+                float dk = alpha[k] * base;
+                double e[GROUP];
+                for (int i = 0; i < GROUP; ++i) {
+                    float qw = fake_quant(w[i], dk);
+                    float ei = w[i] - qw;
+                    e[i] = (double)ei;
+                }
+                double E = 0.0;
+                for (int i = 0; i < GROUP; ++i)
+                    for (int j = 0; j < GROUP; ++j)
+                        E += e[i] * (double)Hg[i * ldh + j] * e[j];
+                if (all_err) all_err[(r * G + g) * K + k] = E;
+                if (best_k < 0 || E < best) {
+                    best = E;
+                    best_k = k;
+                    best_delta = dk;
+                }
+            }
+            delta_out[r * G + g] = best_delta;
+            idx_out[r * G + g] = best_k;
+            best_err[r * G + g] = best;
+        }
+    }
+}
+
+/* ----------------------------------------------------------- (c) LSQ forward
+ * [blog] section 3: the forward pass emulates the deployment INT4 grid,
+ * Q = Delta * clamp(round(w / Delta), -8, 7), each group with its own Delta.
+ * W, Q: float [R, C]; delta: float [R, C/32]. */
+void oracle_lsq_fwd(const float *W, const float *delta, int64_t R, int64_t C, float *Q)
+{
+    const int64_t G = C / GROUP;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t c = 0; c < C; ++c)
+            Q[r * C + c] = fake_quant(W[r * C + c], delta[r * G + c / GROUP]);
+}
+
+/* ---------------------------------------------------------- (c) LSQ backward
+ * [blog] section 3: round is passed straight through (STE) to the weights;
+ * LSQ carries the task gradient to the step size, normalised by the group's
+ * element count and the number of positive levels (s = 1/sqrt(32*7) is
+ * passed in as grad_scale).  With v = w / Delta (the same binary32 value as
+ * the forward):
+ *   grad_W = G            if -8 <= v <= 7, else 0
+ *   dQ/dDelta = rint(v) - v  if -8 < v < 7;  -8 if v <= -8;  7 if v >= 7
+ *   grad_Delta[r, g] = s * sum_{i in g} G_i * dQ_i/dDelta   (sum in double)
+ * G: float [R, C] when g_is_bf16 == 0, else bf16 bits [R, C].
+ * grad_W: float [R, C]; grad_delta: double [R, C/32]. */
+void oracle_lsq_bwd(const float *W, const float *delta, const void *Gp, int g_is_bf16,
+                    int64_t R, int64_t C, float grad_scale,
+                    float *grad_W, double *grad_delta)
+{
+    const int64_t G = C / GROUP;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t g = 0; g < G; ++g) {
+            float dl = delta[r * G + g];
+            double acc = 0.0;
+            for (int i = 0; i < GROUP; ++i) {
+                int64_t idx = r * C + g * GROUP + i;
+                float gi = g_is_bf16 ? bf16_to_float(((const uint16_t *)Gp)[idx])
+                                     : ((const float *)Gp)[idx];
+                float v = scaled(W[idx], dl);
+                int inside = (v >= QMIN) && (v <= QMAX);
+                grad_W[idx] = inside ? gi : 0.0f;
+                float d;
+                if (v <= QMIN)      d = QMIN;
+                else if (v >= QMAX) d = QMAX;
+                else                d = rintf(v) - v;
+                acc += (double)gi * (double)d;
+            }
+            grad_delta[r * G + g] = (double)grad_scale * acc;
+        }
+    }
+}
+
+/* ------------------------------------------------------------ (c) W4A16 pack
+ * [card] "QAT Highlights": the same INT4 grid is used at initialisation, QAT
+ * and export, so the exported codes are the forward codes
+ * q = clamp(rint(w / Delta), -8, 7) with the binary32 Delta.  Element 2j goes
+ * to the low nibble of byte j and element 2j+1 to the high nibble (4-bit
+ * two's complement); the per-group scale is exported as IEEE binary16,
+ * round-to-nearest-even.
+ * packed: uint8 [R, C/2]; scale16: binary16 bits [R, C/32]. */
+void oracle_pack_w4a16(const float *W, const float *delta, int64_t R, int64_t C,
+                       uint8_t *packed, uint16_t *scale16)
+{
+    const int64_t G = C / GROUP;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t j = 0; j < C / 2; ++j) {
+            int64_t c0 = 2 * j, c1 = 2 * j + 1;
+            int lo = (int)code_of(scaled(W[r * C + c0], delta[r * G + c0 / GROUP]));
+            int hi = (int)code_of(scaled(W[r * C + c1], delta[r * G + c1 / GROUP]));
+            packed[r * (C / 2) + j] = (uint8_t)((lo & 0xF) | ((hi & 0xF) << 4));
+        }
+        for (int64_t g = 0; g < G; ++g) {
+            _Float16 h = (_Float16)delta[r * G + g];
+            uint16_t bits;
+            memcpy(&bits, &h, sizeof bits);
+            scale16[r * G + g] = bits;
+        }
+    }
+}
+
+/* Codes only (int8), for unpack checks. */
+void oracle_codes(const float *W, const float *delta, int64_t R, int64_t C, int8_t *codes)
+{
+    const int64_t G = C / GROUP;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t c = 0; c < C; ++c)
+            codes[r * C + c] = (int8_t)code_of(scaled(W[r * C + c], delta[r * G + c / GROUP]));
+}

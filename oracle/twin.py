@@ -1,0 +1,79 @@
+"""Second, independent NumPy statement of the quantizer (tiny inputs only).
+
+TEST INFRASTRUCTURE.  Written separately from ``qat4_oracle.c`` (vectorised
+NumPy instead of C loops) so that the two can be checked against each other on
+small cases.  Same readings of the pages as the C oracle:
+
+* Q_Delta(w) = Delta * clamp(rint(w / Delta), -8, 7) in float32, Delta = 0 -> 0
+  ("Opt.Gear-QAT" blog, section 1 and section 3; model card "Quantization
+  Configuration", symmetric zero-point 0);
+* per-group objective e H_gg e^T over Delta_k = alpha_k * (max|w| / 7) (model
+  card objective, block-diagonal reading);
+* LSQ gradients (blog section 3; Esser et al. 2020).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+f32 = np.float32
+
+
+def _v(w, d):
+    w = np.asarray(w, f32)
+    d = np.asarray(d, f32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = np.where(d == 0, f32(0), w / np.where(d == 0, f32(1), d))
+    return v.astype(f32)
+
+
+def codes(w, d):
+    return np.clip(np.rint(_v(w, d)), f32(-8), f32(7)).astype(f32)
+
+
+def fake_quant(w, d):
+    return (np.asarray(d, f32) * codes(w, d)).astype(f32)
+
+
+def search(W, H, alpha):
+    """Exhaustive grid search; returns (delta, idx, best_err float64, all_err)."""
+    W = np.asarray(W, f32)
+    R, C = W.shape
+    G = C // 32
+    alpha = np.asarray(alpha, f32)
+    K = alpha.size
+    Wg = W.reshape(R, G, 32)
+    m = np.abs(Wg).max(axis=2)                          # [R, G]
+    base = (m / f32(7)).astype(f32)
+    dk = (alpha[None, None, :] * base[:, :, None]).astype(f32)   # [R, G, K]
+    q = fake_quant(Wg[:, :, None, :], dk[:, :, :, None])         # [R, G, K, 32]
+    e = (Wg[:, :, None, :] - q).astype(f32).astype(np.float64)
+    Hb = np.stack([np.asarray(H, np.float64)[32 * g:32 * g + 32, 32 * g:32 * g + 32]
+                   for g in range(G)])                           # [G, 32, 32]
+    E = np.einsum("rgki,gij,rgkj->rgk", e, Hb, e)
+    idx = np.argmin(E, axis=2).astype(np.int32)                  # first minimum
+    best = np.take_along_axis(E, idx[:, :, None].astype(np.int64), axis=2)[:, :, 0]
+    delta = np.take_along_axis(dk, idx[:, :, None].astype(np.int64), axis=2)[:, :, 0]
+    return delta.astype(f32), idx, best, E
+
+
+def lsq_bwd(W, delta, G, s):
+    W = np.asarray(W, f32)
+    R, C = W.shape
+    d = np.repeat(np.asarray(delta, f32), 32, axis=1)
+    v = _v(W, d)
+    G = np.asarray(G, f32)
+    gW = np.where((v >= -8) & (v <= 7), G, f32(0)).astype(f32)
+    dq = np.where(v <= -8, f32(-8), np.where(v >= 7, f32(7), (np.rint(v) - v).astype(f32)))
+    gD = float(s) * (G.astype(np.float64) * dq.astype(np.float64)).reshape(R, C // 32, 32).sum(axis=2)
+    return gW, gD
+
+
+def pack(W, delta):
+    W = np.asarray(W, f32)
+    R, C = W.shape
+    q = codes(W, np.repeat(np.asarray(delta, f32), 32, axis=1)).astype(np.int8)
+    nib = (q.astype(np.int16) & 0xF).astype(np.uint8)
+    packed = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    with np.errstate(over="ignore"):
+        s16 = np.asarray(delta, f32).astype(np.float16).view(np.uint16)
+    return packed, s16
