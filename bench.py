@@ -1,0 +1,439 @@
+"""Benchmark of the group-32 INT4 quantizer path on B200.
+
+One step = one pass of the whole path over one 1B-class MLP up-projection
+(W fp32 8192x2048, calibration X bf16 262144x2048 with 1% outlier channels,
+101-candidate grid, upstream gradient bf16):
+
+    H = hessian(X) -> (delta, idx, err) = scale_search(W, H, alpha)
+      -> (Q, grad_W, grad_delta) = lsq_fwd_bwd(W, delta, G) -> pack_w4a16(W, delta)
+
+Every input is resident in HBM before timing starts.  Before each stage the
+L2 cache (126 MB) is flushed by a read sweep over a 512 MB buffer, so no
+stage reads its inputs from L2; the flushes are inside ms_per_step but not
+inside the per-kernel times.  Per-kernel times are CUDA events on the stream
+the kernels run on.
+
+The headline `value` is the first metric of the path, LSQ fwd+bwd GB/s
+(14.25 algorithmic bytes per weight); the Hessian TFLOP/s, scale-search
+groups/s and pack GB/s are in `stages`, each with its roofline.  With N GPUs
+every rank quantizes its own layer (independent problems, weak scaling, no
+collective on the data path); the value is the bytes of all ranks divided by
+the slowest rank's time.
+
+`--impl reference` times the CPU oracle instead (test infrastructure, run
+only here and in the tests) on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "LSQ fwd+bwd GB/s (% HBM peak); scale-search groups/s; Hessian TFLOP/s"
+LSQ_BYTES_PER_ELT = 14.25       # W 4 + G(bf16) 2 + Q 4 + grad_W 4 + (delta 4 + grad_delta 4)/32
+PACK_BYTES_PER_ELT = 4.6875     # W 4 + delta 4/32 + nibbles 0.5 + fp16 scale 2/32
+SEARCH_OPS_PER_CAND = 720       # 528 FMA quadratic form + 32 x (div, rint, min, max, mul, sub)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+# --------------------------------------------------------------------------- setup
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def layer_seed(rank: int) -> int:
+    """Every rank quantizes its own, independently seeded layer."""
+    return rank
+
+
+def aggregate_over_ranks(local_units: float, local_ms: float, group=None):
+    """(sum of units over ranks, max of ms over ranks); plain values when not distributed."""
+    import torch
+    import torch.distributed as dist
+    if group is None and not (dist.is_available() and dist.is_initialized()):
+        return float(local_units), float(local_ms)
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend(group) == "nccl" else "cpu"
+    u = torch.tensor([local_units], dtype=torch.float64, device=dev)
+    t = torch.tensor([local_ms], dtype=torch.float64, device=dev)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM, group=group)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(u.item()), float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples during the timed region."""
+
+    def __init__(self, index: int, out_path: str | None = None):
+        self.index = index
+        self.proc = None
+        self.out_path = out_path
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={CLOCK_FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            if self.out_path:
+                with open(self.out_path, "w") as fh:
+                    fh.write(CLOCK_FIELDS + "\n" + "\n".join(self.lines) + "\n")
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, val in zip(names, f[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        load = [s for s in sm if s > 500] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------ our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import int4_group_wise_b200 as q4
+    from int4_group_wise_b200 import inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    peaks, peak_kind = load_peaks()
+
+    wl = inputs.workload(args.config)
+    m = wl.matrices[0]
+    seed = layer_seed(rank)
+    t0 = time.time()
+    W_h = wl.weight(m, seed)
+    X_h = wl.activations(m.x_name, seed)
+    G_h = wl.grad(m, seed)
+    alpha_h = wl.alpha()
+    gen_s = time.time() - t0
+    R, C = W_h.shape
+    n = X_h.shape[0]
+    groups = R * C // 32
+    K = alpha_h.size
+
+    # pinned host copies (for the end-to-end leg) and device-resident inputs
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    W_p, X_p, G_p, a_p = pin(W_h), pin(X_h.view(np.int16)), pin(G_h.view(np.int16)), pin(alpha_h)
+    W = W_p.to(dev)
+    X = X_p.to(dev).view(torch.bfloat16)
+    G = G_p.to(dev).view(torch.bfloat16)
+    alpha = a_p.to(dev)
+    H = torch.empty((C, C), dtype=torch.float32, device=dev)
+    ws_bytes = q4.hessian_workspace_bytes(n, C)
+    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
+    delta = torch.empty((R, C // 32), dtype=torch.float32, device=dev)
+    idx = torch.empty((R, C // 32), dtype=torch.int32, device=dev)
+    err = torch.empty((R, C // 32), dtype=torch.float32, device=dev)
+    Q = torch.empty_like(W)
+    gW = torch.empty_like(W)
+    gD = torch.empty_like(delta)
+    packed = torch.empty((R, C // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((R, C // 32), dtype=torch.float16, device=dev)
+    flush_buf = torch.ones(128 << 20, dtype=torch.float32, device=dev)   # 512 MB
+    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def flush():
+        torch.sum(flush_buf, dim=0, out=flush_sink)
+
+    stages = ["hessian", "scale_search", "lsq_fwd_bwd", "pack_w4a16"]
+
+    def step(ev=None):
+        def run(i, fn):
+            flush()
+            if ev is not None:
+                ev[i][0].record(stream)
+            fn()
+            if ev is not None:
+                ev[i][1].record(stream)
+        run(0, lambda: q4.hessian(X, H, ws))
+        run(1, lambda: q4.scale_search(W, H, alpha, delta, idx, err))
+        run(2, lambda: q4.lsq_fwd_bwd(W, delta, G, q4.GRAD_SCALE, Q, gW, gD))
+        run(3, lambda: q4.pack_w4a16(W, delta, packed, scales))
+
+    for _ in range(args.warmup):
+        step()
+    q4.sync_check()
+
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in stages] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"bench_clocks_r{rank}.csv")) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    q4.sync_check()
+    total_ms = start.elapsed_time(stop)
+    per = {s: [evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(args.steps)] for i, s in enumerate(stages)}
+    mean = {s: sum(v) / len(v) for s, v in per.items()}
+
+    # ---- end-to-end leg: the lsq_fwd_bwd call from pinned host memory and back
+    Q_p = torch.empty(Q.shape, dtype=Q.dtype).pin_memory()
+    gW_p = torch.empty(gW.shape, dtype=gW.dtype).pin_memory()
+    gD_p = torch.empty(gD.shape, dtype=gD.dtype).pin_memory()
+    d_p = delta.cpu().pin_memory()
+    W2, G2, d2 = torch.empty_like(W), torch.empty_like(G), torch.empty_like(delta)
+
+    def e2e_step():
+        W2.copy_(W_p, non_blocking=True)
+        G2.copy_(G_p.view(torch.bfloat16), non_blocking=True)
+        d2.copy_(d_p, non_blocking=True)
+        q4.lsq_fwd_bwd(W2, d2, G2, q4.GRAD_SCALE, Q, gW, gD)
+        Q_p.copy_(Q, non_blocking=True)
+        gW_p.copy_(gW, non_blocking=True)
+        gD_p.copy_(gD, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e2e_n = max(3, min(args.steps, 10))
+    a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a_.record(stream)
+    for _ in range(e2e_n):
+        e2e_step()
+    b_.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a_.elapsed_time(b_) / e2e_n
+    h2d = W.numel() * 4 + G.numel() * 2 + delta.numel() * 4
+    d2h = Q.numel() * 4 + gW.numel() * 4 + gD.numel() * 4
+
+    # ---- whole-job aggregation (max time over ranks)
+    lsq_bytes = LSQ_BYTES_PER_ELT * R * C
+    job_lsq_bytes, job_lsq_ms = aggregate_over_ranks(lsq_bytes, mean["lsq_fwd_bwd"])
+    job_step_units, job_total_ms = aggregate_over_ranks(1.0, total_ms)
+    job_e2e_bytes, job_e2e_ms = aggregate_over_ranks(lsq_bytes, e2e_ms)
+    job_h_flop, job_h_ms = aggregate_over_ranks(float(n) * C * (C + 1), mean["hessian"])
+    job_groups, job_s_ms = aggregate_over_ranks(float(groups), mean["scale_search"])
+    job_pack_bytes, job_p_ms = aggregate_over_ranks(PACK_BYTES_PER_ELT * R * C, mean["pack_w4a16"])
+
+    if rank == 0:
+        clocks = clk.summary()
+        hbm = float(peaks["hbm_gbs"])
+        tc_peak = float(peaks["bf16_tflops"])
+        sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+        fp32_ops_peak = 148 * 128 * sm_max * 1e6            # one FP32 op per lane per clock
+        search_roof = fp32_ops_peak / (SEARCH_OPS_PER_CAND * K)   # groups/s, one GPU
+        lsq_gbs = job_lsq_bytes / job_lsq_ms / 1e6
+        stage_lines = {
+            "hessian": {"value": job_h_flop / job_h_ms / 1e9, "unit": "TFLOP/s", "ms": mean["hessian"],
+                        "roofline": {"bound": "tensor", "peak": tc_peak * world, "unit": "TFLOP/s",
+                                     "frac": job_h_flop / job_h_ms / 1e9 / (tc_peak * world),
+                                     "algorithmic_per_launch": float(n) * C * (C + 1),
+                                     "peak_kind": f"{peak_kind} bf16 burst"}},
+            "scale_search": {"value": job_groups / job_s_ms * 1e3, "unit": "groups/s", "ms": mean["scale_search"],
+                             "roofline": {"bound": "alu", "peak": search_roof * world, "unit": "groups/s",
+                                          "frac": job_groups / job_s_ms * 1e3 / (search_roof * world),
+                                          "ops_per_group": SEARCH_OPS_PER_CAND * K,
+                                          "peak_kind": f"148 SM x 128 FP32 lanes x {sm_max:.0f} MHz"}},
+            "lsq_fwd_bwd": {"value": lsq_gbs, "unit": "GB/s", "ms": mean["lsq_fwd_bwd"],
+                            "roofline": {"bound": "hbm", "peak": hbm * world, "unit": "GB/s",
+                                         "frac": lsq_gbs / (hbm * world), "bytes_per_launch": lsq_bytes,
+                                         "peak_kind": f"{peak_kind} copy"}},
+            "pack_w4a16": {"value": job_pack_bytes / job_p_ms / 1e6, "unit": "GB/s", "ms": mean["pack_w4a16"],
+                           "roofline": {"bound": "hbm", "peak": hbm * world, "unit": "GB/s",
+                                        "frac": job_pack_bytes / job_p_ms / 1e6 / (hbm * world),
+                                        "bytes_per_launch": PACK_BYTES_PER_ELT * R * C,
+                                        "peak_kind": f"{peak_kind} copy"}},
+        }
+        dominant = max(stages, key=lambda s: mean[s])
+        dom = stage_lines[dominant]["roofline"]
+        if dominant == "hessian":
+            achieved, dom_peak = job_h_flop / job_h_ms / 1e9 / world, tc_peak
+        elif dominant == "scale_search":
+            achieved, dom_peak = job_groups / job_s_ms * 1e3 * SEARCH_OPS_PER_CAND * K / 1e12 / world, \
+                fp32_ops_peak / 1e12
+        else:
+            achieved = stage_lines[dominant]["value"] / world
+            dom_peak = hbm
+        roof_unit = {"hessian": "TFLOP/s", "scale_search": "Top/s"}.get(dominant, "GB/s")
+        line = {
+            "metric": METRIC, "value": lsq_gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": job_total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "1B-class MLP up-projection: W fp32 8192x2048, X bf16 262144x2048 "
+                                   "(1% outlier channels x20), 101-candidate grid, G bf16",
+                       "config_index": args.config, "R": R, "C": C, "n_calib": n, "K": K,
+                       "parallelism": f"replicas x{world} (one layer per GPU)",
+                       "l2": "flushed (512 MB read sweep) before every stage; flush time in ms_per_step only"},
+            "roofline": {"kernel": dominant, "bound": dom["bound"], "achieved": achieved, "peak": dom_peak,
+                         "unit": roof_unit, "frac": achieved / dom_peak,
+                         "traffic": None, "peak_kind": dom["peak_kind"]},
+            "stages": stage_lines,
+            "e2e": {"value": job_e2e_bytes / job_e2e_ms / 1e6, "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "what": "lsq_fwd_bwd from pinned host W, G, delta and back to pinned host Q, grad_W, grad_delta"},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clocks,
+            "input_gen_s": round(gen_s, 1),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(W_h, X_h, G_h, alpha_h)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------------ CPU oracle legs
+def _oracle_sample(W, X, G, alpha, rows: int, hblocks: int):
+    """One bounded sample of the step on the CPU oracle; returns per-stage (units, seconds)."""
+    import oracle
+    from int4_group_wise_b200.inputs import bf16_bits_to_f32  # noqa: F401  (inputs only)
+    res = {}
+    Ws, Gs = W[:rows], G[:rows]
+    C = W.shape[1]
+    t = time.perf_counter()
+    Hd = np.zeros((C, C), np.float32)
+    for g in range(hblocks):
+        Hd[32 * g:32 * g + 32, 32 * g:32 * g + 32] = oracle.hessian_block(X, 32 * g, 32, 32 * g, 32)
+    res["hessian"] = (float(X.shape[0]) * 32 * 33 * hblocks, time.perf_counter() - t)
+    Wsearch = Ws[:, :32 * hblocks]
+    t = time.perf_counter()
+    d, i, b = oracle.scale_search(Wsearch, Hd[:32 * hblocks, :32 * hblocks], alpha)
+    res["scale_search"] = (float(Wsearch.size // 32), time.perf_counter() - t)
+    delta = (np.abs(Ws).reshape(rows, -1, 32).max(axis=2) / np.float32(7)).astype(np.float32)
+    t = time.perf_counter()
+    oracle.lsq_fwd(Ws, delta)
+    oracle.lsq_bwd(Ws, delta, Gs, float(np.float32(1 / np.sqrt(224))))
+    res["lsq_fwd_bwd"] = (LSQ_BYTES_PER_ELT * Ws.size, time.perf_counter() - t)
+    t = time.perf_counter()
+    oracle.pack_w4a16(Ws, delta)
+    res["pack_w4a16"] = (PACK_BYTES_PER_ELT * Ws.size, time.perf_counter() - t)
+    return res
+
+
+def cpu_baseline(W, X, G, alpha, rows=2048, hblocks=8):
+    import oracle
+    cores = oracle.set_threads(0)
+    res = _oracle_sample(W, X, G, alpha, rows, hblocks)
+    u, s = res["lsq_fwd_bwd"]
+    return {"value": u / s / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"rows 0..{rows - 1} of W for LSQ/pack ({rows}x{W.shape[1]}); "
+                      f"{hblocks} diagonal 32x32 Hessian blocks over all {X.shape[0]} rows; "
+                      f"scale search on those {hblocks} groups x {rows} rows",
+            "stages": {"hessian_gflops": res["hessian"][0] * 1e-9 / res["hessian"][1] * 1.0,
+                       "scale_search_groups_per_s": res["scale_search"][0] / res["scale_search"][1],
+                       "lsq_fwd_bwd_gbs": u / s / 1e9,
+                       "pack_w4a16_gbs": res["pack_w4a16"][0] / res["pack_w4a16"][1] / 1e9}}
+
+
+def run_reference(args):
+    """The oracle as it stands, on the host cores, on bounded samples of the same workload."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    from int4_group_wise_b200 import inputs
+    wl = inputs.workload(args.config)
+    m = wl.matrices[0]
+    W, G, alpha = wl.weight(m), wl.grad(m), wl.alpha()
+    X = wl.activations(m.x_name, n=16384)          # a row sample of the calibration set
+    cores = oracle.set_threads(0)
+    rows = 512
+    for _ in range(args.warmup):
+        _oracle_sample(W, X, G, alpha, rows, 2)
+    tot_u = tot_s = 0.0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        r = _oracle_sample(W, X, G, alpha, rows, 2)
+        tot_u += r["lsq_fwd_bwd"][0]
+        tot_s += r["lsq_fwd_bwd"][1]
+    wall = time.perf_counter() - t0
+    v = tot_u / tot_s / 1e9
+    sample = (f"per step: rows 0..{rows - 1} of W (LSQ, pack); 2 diagonal Hessian blocks over 16384 "
+              f"calibration rows; scale search on 2 groups x {rows} rows")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": wall * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": "1B-class MLP up-projection (CPU oracle, row sample)", "config_index": args.config},
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

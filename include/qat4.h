@@ -1,0 +1,182 @@
+/*
+ * qat4.h -- C ABI of libqat4, a B200 (sm_100a) implementation of the
+ * group-32 symmetric INT4 weight quantizer used for quantization-aware
+ * training with a W4A16 export:
+ *
+ *   (a) calibration Hessian            H = X^T X / n
+ *   (b) Hessian-weighted scale search  Delta* = argmin over a grid of
+ *                                      e H_gg e^T, e = w_g - Q_Delta(w_g)
+ *   (c) LSQ fake-quant forward         Q = Delta * clamp(rint(w / Delta), -8, 7)
+ *       LSQ backward                   straight-through grad to W, step grad to Delta
+ *       W4A16 export                   4-bit codes + binary16 scales
+ *
+ * Sources: the model card "Opt.Gear-1B-qat-int4-per-channel-unquantized"
+ * (section "Quantization Configuration": symmetric INT4 with zero-point 0,
+ * and the per-group objective Delta* = argmin ||W X - Q_Delta(W) X||_F^2;
+ * section "QAT Highlights": group size 32 and one grid for initialisation,
+ * QAT and export) and the blog post "Opt.Gear-QAT: Preserving On-Device
+ * Performance with QAT" (section "Quantization parameters of Opt.Gear-1B":
+ * one scale per 32 weights; section 2 "Hessian-based scale initialize";
+ * section 3 "LSQ-based QAT").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Data pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates device or host memory and keeps no per-call state.
+ *  - Matrices are row-major and dense (row stride = number of columns)
+ *    unless a leading dimension is given.  A weight matrix W is [R, C]
+ *    (R output rows, C input columns); group (r, g) is W[r, 32g : 32g+32],
+ *    so C must be a positive multiple of 32.  Per-group arrays are
+ *    [R, C/32] row-major.
+ *  - Every call is asynchronous on `stream` (0 = legacy default stream).
+ *    Argument errors are detected on the host before anything is launched
+ *    and nothing is written; launch failures return QAT4_ERR_CUDA.
+ *  - Pointers must be 16-byte aligned (QAT4_ERR_ALIGN otherwise).
+ *  - Inputs are assumed finite.  Delta = 0 is allowed (it only arises for an
+ *    all-zero group): such a group quantizes to 0, its weight gradient is G
+ *    and its step gradient is 0.
+ *  - Rounding: w / Delta is an IEEE binary32 division, round() is
+ *    round-half-to-even, Delta * q is one binary32 multiply; integer codes,
+ *    Q, grad_W and packed bytes are therefore exactly reproducible.
+ */
+#ifndef QAT4_H
+#define QAT4_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    QAT4_OK = 0,
+    QAT4_ERR_NULL = 1,       /* a required pointer is NULL */
+    QAT4_ERR_SHAPE = 2,      /* R, C, n or K out of range, C % 32 != 0, ldh < C */
+    QAT4_ERR_ALIGN = 3,      /* a pointer is not 16-byte aligned */
+    QAT4_ERR_DTYPE = 4,      /* unknown qat4_dtype */
+    QAT4_ERR_WORKSPACE = 5,  /* workspace missing or smaller than required */
+    QAT4_ERR_CUDA = 6,       /* a CUDA runtime/driver call or a launch failed */
+    QAT4_ERR_TIMEOUT = 7     /* a kernel gave up a bounded wait (see qat4_sync_check) */
+} qat4_status;
+
+typedef enum { QAT4_F32 = 0, QAT4_BF16 = 1 } qat4_dtype;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+const char *qat4_status_string(qat4_status status);
+
+/* ABI version of this header (incremented on incompatible changes). */
+int qat4_abi_version(void);
+
+/* ---------------------------------------------------------------- (a)
+ * Calibration Hessian H = X^T X / n  (blog section 2: layer sensitivity
+ * from calibration inputs, the second-order output-reconstruction view).
+ *
+ *  X          bf16 bit patterns, [n, C] row-major (n calibration tokens).
+ *  n          1 <= n <= 2^31 - 1.
+ *  C          number of input channels, multiple of 32, 32 <= C <= 65536.
+ *  H          float32 [C, C] row-major, written in full (both triangles,
+ *             bitwise symmetric).  Products are exact, sums are float32 on
+ *             the tensor cores (bf16 x bf16 -> fp32), scaled by 1/n.
+ *  workspace  device scratch of at least qat4_hessian_workspace_bytes(n, C)
+ *             bytes (may be NULL when that is 0); contents on entry are
+ *             ignored.  The result does not depend on the device's SM count.
+ *  Errors: QAT4_ERR_NULL, _SHAPE, _ALIGN, _WORKSPACE, _CUDA.  A bounded
+ *  wait that gives up inside the kernel is reported by qat4_sync_check.
+ */
+size_t qat4_hessian_workspace_bytes(int64_t n, int64_t C);
+qat4_status qat4_hessian(const uint16_t *X, int64_t n, int64_t C, float *H,
+                         void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* ---------------------------------------------------------------- (b)
+ * Hessian-weighted per-group scale search (model card, "Quantization
+ * Configuration": Delta* = argmin ||W X - Q_Delta(W) X||_F^2 per group,
+ * read block-diagonally: each group minimises e H_gg e^T with the other
+ * groups at zero error; blog section 2).
+ *
+ *  W         float32 [R, C].
+ *  H         float32, row stride ldh >= C; only the C/32 diagonal 32x32
+ *            blocks H[32g:32g+32, 32g:32g+32] are read.  H must be
+ *            symmetric positive semi-definite for the exact-argmin
+ *            guarantee below (any Hessian from qat4_hessian is).
+ *  alpha     float32 [K], K >= 1: candidate multipliers.  Candidate k of
+ *            group (r, g) is Delta_k = fl(alpha[k] * fl(max|w_g| / 7)).
+ *  delta     out float32 [R, C/32]: the chosen Delta_k.
+ *  idx       out int32   [R, C/32]: the chosen k (smallest k on exact ties).
+ *  best_err  out float32 [R, C/32] (may be NULL): e H_gg e^T at the chosen k,
+ *            rounded to float32 from a float64 evaluation.
+ *  Every candidate is screened in float32 with a rigorous rounding-error
+ *  bound; the candidates that the bound cannot separate from the minimum
+ *  are re-scored in float64, so idx equals the argmin of the float64
+ *  objective except for candidates whose objectives agree to ~1e-15.
+ *  Errors: QAT4_ERR_NULL, _SHAPE, _ALIGN, _CUDA.
+ */
+qat4_status qat4_scale_search(const float *W, int64_t R, int64_t C,
+                              const float *H, int64_t ldh,
+                              const float *alpha, int32_t K,
+                              float *delta, int32_t *idx, float *best_err,
+                              cudaStream_t stream);
+
+/* ---------------------------------------------------------------- (c)
+ * LSQ fake-quant forward (blog section 3: the forward pass emulates the
+ * deployment INT4 grid):  Q = Delta * clamp(rint(w / Delta), -8, 7).
+ *
+ *  W      float32 [R, C];  delta float32 [R, C/32];  Q out float32 [R, C].
+ *  Errors: QAT4_ERR_NULL, _SHAPE, _ALIGN, _CUDA.
+ */
+qat4_status qat4_lsq_fwd(const float *W, const float *delta, int64_t R, int64_t C,
+                         float *Q, cudaStream_t stream);
+
+/* LSQ backward (blog section 3: straight-through estimator for round; the
+ * step-size gradient normalised by the group's element count and the
+ * number of positive levels; Esser et al., "Learned Step Size
+ * Quantization", ICLR 2020).  With v = w / Delta:
+ *    grad_W     = G                       if -8 <= v <= 7, else 0
+ *    dQ/dDelta  = rint(v) - v             if -8 <  v <  7
+ *               = -8 if v <= -8,  7 if v >= 7
+ *    grad_delta = grad_scale * sum over the group of G * dQ/dDelta
+ *  G           [R, C], float32 (QAT4_F32) or bf16 bit patterns (QAT4_BF16).
+ *  grad_scale  normally 1/sqrt(32 * 7).
+ *  grad_W      out float32 [R, C];  grad_delta out float32 [R, C/32]
+ *              (overwritten, not accumulated).
+ *  Errors: QAT4_ERR_NULL, _SHAPE, _ALIGN, _DTYPE, _CUDA.
+ */
+qat4_status qat4_lsq_bwd(const float *W, const float *delta, const void *G, qat4_dtype g_dtype,
+                         int64_t R, int64_t C, float grad_scale,
+                         float *grad_W, float *grad_delta, cudaStream_t stream);
+
+/* Forward and backward in one pass over W and G (the outputs of
+ * qat4_lsq_fwd and qat4_lsq_bwd, bit-identical Q and grad_W). */
+qat4_status qat4_lsq_fwd_bwd(const float *W, const float *delta, const void *G, qat4_dtype g_dtype,
+                             int64_t R, int64_t C, float grad_scale,
+                             float *Q, float *grad_W, float *grad_delta, cudaStream_t stream);
+
+/* W4A16 export (model card, "QAT Highlights": the same INT4 grid at
+ * initialisation, QAT and export).  Codes are the forward codes
+ * clamp(rint(w / Delta), -8, 7) for the float32 Delta.
+ *
+ *  packed  out uint8 [R, C/2]: byte j of a row holds element 2j in its low
+ *          nibble and element 2j+1 in its high nibble (4-bit two's complement).
+ *  scales  out binary16 bit patterns [R, C/32]: Delta rounded to nearest even.
+ *  Errors: QAT4_ERR_NULL, _SHAPE, _ALIGN, _CUDA.
+ */
+qat4_status qat4_pack_w4a16(const float *W, const float *delta, int64_t R, int64_t C,
+                            uint8_t *packed, uint16_t *scales, cudaStream_t stream);
+
+/* Synchronises `stream`, then reads and clears the library's device error
+ * word for the current device.  Returns QAT4_ERR_TIMEOUT if a kernel gave up
+ * a bounded wait since the last check, QAT4_ERR_CUDA if synchronisation
+ * failed, QAT4_OK otherwise. */
+qat4_status qat4_sync_check(cudaStream_t stream);
+
+/* Exercises the bounded-wait path: launches one tiny kernel that waits on a
+ * barrier which nothing ever completes, for at most limit_ns nanoseconds
+ * (1 <= limit_ns <= 10^10), after which it records a timeout in the device
+ * error word and returns.  qat4_sync_check then returns QAT4_ERR_TIMEOUT. */
+qat4_status qat4_selftest_bounded_wait(int64_t limit_ns, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* QAT4_H */

@@ -1,0 +1,285 @@
+// qat4_api.cu -- the C ABI of libqat4 (declared in include/qat4.h): argument
+// validation on the host, launch configuration, and the device error word.
+// All kernels live in the headers included below; this is the only
+// translation unit of the library.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/qat4.h"
+#include "device_common.cuh"
+#include "hessian.cuh"
+#include "lsq_pack.cuh"
+#include "scale_search.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool valid_rc(int64_t R, int64_t C) {
+    return R >= 1 && C >= 32 && (C % 32) == 0 && R <= (int64_t(1) << 31) - 1 &&
+           C <= (int64_t(1) << 31) - 1 && R * C <= (int64_t(1) << 40);
+}
+
+struct DeviceInfo {
+    int sms = 0;
+    bool hessian_attr = false;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mutex;
+
+// Current device and its SM count (cached); false on any CUDA error.
+bool device_info(int* dev_out, DeviceInfo** info) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceInfo& d = g_dev[dev];
+    if (d.sms == 0) {
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+            return false;
+        d.sms = sms;
+    }
+    *dev_out = dev;
+    *info = &d;
+    return true;
+}
+
+qat4_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? QAT4_OK : QAT4_ERR_CUDA;
+}
+
+// Blocks for a grid-stride streaming kernel over `nquads` float4 quads:
+// enough warps to cover the work once, at most 8 resident blocks per SM.
+unsigned stream_blocks(int64_t nquads, int sms, int unroll) {
+    const int64_t warp_steps = (nquads + 31) / 32;
+    const int64_t warps_needed = (warp_steps + unroll - 1) / unroll;
+    const int64_t blocks_needed = (warps_needed + (qat4::kStreamThreads / 32) - 1) / (qat4::kStreamThreads / 32);
+    const int64_t cap = static_cast<int64_t>(sms) * (2048 / qat4::kStreamThreads);
+    return static_cast<unsigned>(std::max<int64_t>(1, std::min(blocks_needed, cap)));
+}
+
+// --------------------------------------------------------------- tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static std::once_flag once;
+    static EncodeTiledFn fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* qat4_status_string(qat4_status s) {
+    switch (s) {
+        case QAT4_OK: return "QAT4_OK";
+        case QAT4_ERR_NULL: return "QAT4_ERR_NULL: a required pointer is NULL";
+        case QAT4_ERR_SHAPE: return "QAT4_ERR_SHAPE: size out of range or C not a multiple of 32";
+        case QAT4_ERR_ALIGN: return "QAT4_ERR_ALIGN: pointer not 16-byte aligned";
+        case QAT4_ERR_DTYPE: return "QAT4_ERR_DTYPE: unknown gradient dtype";
+        case QAT4_ERR_WORKSPACE: return "QAT4_ERR_WORKSPACE: workspace missing or too small";
+        case QAT4_ERR_CUDA: return "QAT4_ERR_CUDA: a CUDA call or kernel launch failed";
+        case QAT4_ERR_TIMEOUT: return "QAT4_ERR_TIMEOUT: a kernel gave up a bounded wait";
+    }
+    return "QAT4_ERR_UNKNOWN";
+}
+
+int qat4_abi_version(void) { return 1; }
+
+// ------------------------------------------------------------------ Hessian
+size_t qat4_hessian_workspace_bytes(int64_t n, int64_t C) {
+    (void)n;
+    (void)C;
+    return 0;   // one CTA per output tile: no split-reduction scratch
+}
+
+qat4_status qat4_hessian(const uint16_t* X, int64_t n, int64_t C, float* H,
+                         void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (!X || !H) return QAT4_ERR_NULL;
+    if (n < 1 || n > (int64_t(1) << 31) - 1 || C < 32 || C % 32 != 0 || C > 65536) return QAT4_ERR_SHAPE;
+    if (!aligned16(X) || !aligned16(H)) return QAT4_ERR_ALIGN;
+    if (workspace_bytes < qat4_hessian_workspace_bytes(n, C)) return QAT4_ERR_WORKSPACE;
+    (void)workspace;
+
+    int dev;
+    DeviceInfo* info;
+    if (!device_info(&dev, &info)) return QAT4_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!info->hessian_attr) {
+            if (cudaFuncSetAttribute(qat4::hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(qat4::kHSmemBytes)) != cudaSuccess)
+                return QAT4_ERR_CUDA;
+            info->hessian_attr = true;
+        }
+    }
+    EncodeTiledFn encode = encode_tiled();
+    if (!encode) return QAT4_ERR_CUDA;
+
+    CUtensorMap tmap;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(n)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(C) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(qat4::kHBK)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return QAT4_ERR_CUDA;
+
+    qat4::HessParams p;
+    p.n = n;
+    p.C = static_cast<int>(C);
+    p.nb = static_cast<int>((C + qat4::kHBM - 1) / qat4::kHBM);
+    p.kblocks = static_cast<int>((n + qat4::kHBK - 1) / qat4::kHBK);
+    p.inv_n = static_cast<float>(1.0 / static_cast<double>(n));
+    // generous bound: 4 s plus 100 ns per calibration row (a tile's mainloop
+    // takes ~2 ns per row at full rate)
+    p.limit_ns = 4000000000ull + 100ull * static_cast<uint64_t>(n);
+    const unsigned tiles = static_cast<unsigned>(p.nb) * (p.nb + 1) / 2;
+    qat4::hessian_tc_kernel<<<tiles, qat4::kHThreads, qat4::kHSmemBytes, stream>>>(tmap, p, H);
+    return launch_status();
+}
+
+// -------------------------------------------------------------- scale search
+qat4_status qat4_scale_search(const float* W, int64_t R, int64_t C, const float* H, int64_t ldh,
+                              const float* alpha, int32_t K, float* delta, int32_t* idx,
+                              float* best_err, cudaStream_t stream) {
+    if (!W || !H || !alpha || !delta || !idx) return QAT4_ERR_NULL;
+    if (!valid_rc(R, C) || K < 1 || ldh < C || C / 32 > 65535) return QAT4_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(H) || !aligned16(alpha) || !aligned16(delta) || !aligned16(idx) ||
+        (best_err && !aligned16(best_err)) || (ldh % 4) != 0)
+        return QAT4_ERR_ALIGN;
+    const dim3 grid(static_cast<unsigned>((R + qat4::kSearchThreads - 1) / qat4::kSearchThreads),
+                    static_cast<unsigned>(C / 32));
+    qat4::scale_search_kernel<<<grid, qat4::kSearchThreads, 0, stream>>>(
+        W, static_cast<int>(R), static_cast<int>(C), H, ldh, alpha, K, delta, idx, best_err);
+    return launch_status();
+}
+
+// ---------------------------------------------------------------------- LSQ
+static qat4_status lsq_common(const float* W, const float* delta, const void* G, qat4_dtype g_dtype,
+                              int64_t R, int64_t C, float grad_scale, float* Q, float* grad_W,
+                              float* grad_delta, bool fwd, bool bwd, cudaStream_t stream) {
+    if (!W || !delta || (fwd && !Q) || (bwd && (!G || !grad_W || !grad_delta))) return QAT4_ERR_NULL;
+    if (!valid_rc(R, C)) return QAT4_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(delta) || (fwd && !aligned16(Q)) ||
+        (bwd && (!aligned16(G) || !aligned16(grad_W) || !aligned16(grad_delta))))
+        return QAT4_ERR_ALIGN;
+    if (bwd && g_dtype != QAT4_F32 && g_dtype != QAT4_BF16) return QAT4_ERR_DTYPE;
+    int dev;
+    DeviceInfo* info;
+    if (!device_info(&dev, &info)) return QAT4_ERR_CUDA;
+    const int64_t nquads = R * C / 4;
+    const unsigned blocks = stream_blocks(nquads, info->sms, qat4::kUnroll);
+    const unsigned th = qat4::kStreamThreads;
+    if (fwd && !bwd) {
+        qat4::lsq_kernel<float, true, false><<<blocks, th, 0, stream>>>(W, delta, nullptr, nquads, 0.f, Q,
+                                                                       nullptr, nullptr);
+    } else if (g_dtype == QAT4_F32) {
+        const float* g = static_cast<const float*>(G);
+        if (fwd)
+            qat4::lsq_kernel<float, true, true><<<blocks, th, 0, stream>>>(W, delta, g, nquads, grad_scale, Q,
+                                                                          grad_W, grad_delta);
+        else
+            qat4::lsq_kernel<float, false, true><<<blocks, th, 0, stream>>>(W, delta, g, nquads, grad_scale,
+                                                                           nullptr, grad_W, grad_delta);
+    } else {
+        const uint16_t* g = static_cast<const uint16_t*>(G);
+        if (fwd)
+            qat4::lsq_kernel<uint16_t, true, true><<<blocks, th, 0, stream>>>(W, delta, g, nquads, grad_scale,
+                                                                             Q, grad_W, grad_delta);
+        else
+            qat4::lsq_kernel<uint16_t, false, true><<<blocks, th, 0, stream>>>(W, delta, g, nquads, grad_scale,
+                                                                              nullptr, grad_W, grad_delta);
+    }
+    return launch_status();
+}
+
+qat4_status qat4_lsq_fwd(const float* W, const float* delta, int64_t R, int64_t C, float* Q,
+                         cudaStream_t stream) {
+    return lsq_common(W, delta, nullptr, QAT4_F32, R, C, 0.f, Q, nullptr, nullptr, true, false, stream);
+}
+
+qat4_status qat4_lsq_bwd(const float* W, const float* delta, const void* G, qat4_dtype g_dtype, int64_t R,
+                         int64_t C, float grad_scale, float* grad_W, float* grad_delta,
+                         cudaStream_t stream) {
+    return lsq_common(W, delta, G, g_dtype, R, C, grad_scale, nullptr, grad_W, grad_delta, false, true,
+                      stream);
+}
+
+qat4_status qat4_lsq_fwd_bwd(const float* W, const float* delta, const void* G, qat4_dtype g_dtype,
+                             int64_t R, int64_t C, float grad_scale, float* Q, float* grad_W,
+                             float* grad_delta, cudaStream_t stream) {
+    return lsq_common(W, delta, G, g_dtype, R, C, grad_scale, Q, grad_W, grad_delta, true, true, stream);
+}
+
+// --------------------------------------------------------------------- pack
+qat4_status qat4_pack_w4a16(const float* W, const float* delta, int64_t R, int64_t C, uint8_t* packed,
+                            uint16_t* scales, cudaStream_t stream) {
+    if (!W || !delta || !packed || !scales) return QAT4_ERR_NULL;
+    if (!valid_rc(R, C)) return QAT4_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(delta) || !aligned16(packed) || !aligned16(scales)) return QAT4_ERR_ALIGN;
+    int dev;
+    DeviceInfo* info;
+    if (!device_info(&dev, &info)) return QAT4_ERR_CUDA;
+    const int64_t nquads = R * C / 4;
+    qat4::pack_w4a16_kernel<<<stream_blocks(nquads, info->sms, 4), qat4::kStreamThreads, 0, stream>>>(
+        W, delta, nquads, reinterpret_cast<uint16_t*>(packed), scales);
+    return launch_status();
+}
+
+// ------------------------------------------------------------ error handling
+qat4_status qat4_sync_check(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return QAT4_ERR_CUDA;
+    int word = 0;
+    if (cudaMemcpyFromSymbol(&word, qat4::g_dev_error, sizeof word) != cudaSuccess) return QAT4_ERR_CUDA;
+    if (word != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(qat4::g_dev_error, &zero, sizeof zero) != cudaSuccess) return QAT4_ERR_CUDA;
+        if (word & qat4::QAT4_DEV_ERR_TIMEOUT) return QAT4_ERR_TIMEOUT;
+    }
+    return QAT4_OK;
+}
+
+}  // extern "C"
+
+namespace qat4 {
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // nothing ever arrives on `bar`: the wait runs into its limit and returns
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, limit_ns);
+}
+}  // namespace qat4
+
+extern "C" qat4_status qat4_selftest_bounded_wait(int64_t limit_ns, cudaStream_t stream) {
+    if (limit_ns < 1 || limit_ns > 10000000000ll) return QAT4_ERR_SHAPE;
+    qat4::bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(limit_ns));
+    return launch_status();
+}

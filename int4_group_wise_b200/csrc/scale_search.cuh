@@ -1,0 +1,287 @@
+// scale_search.cuh -- Hessian-weighted per-group scale search.
+//
+// Model card "Opt.Gear-1B-qat-int4-per-channel-unquantized", section
+// "Quantization Configuration": the scale of every quantization group is
+// initialised by minimising the layer-output reconstruction error
+// ||W X - Q_Delta(W) X||^2.  Read block-diagonally, group (r, g) minimises
+// E(Delta) = e H_gg e^T with e = w_g - Q_Delta(w_g) and H_gg the 32x32 diagonal
+// block of H, over the candidates Delta_k = fl(alpha_k * fl(max|w_g| / 7)).
+//
+// Mapping: one CTA = one column group g x 128 rows; thread t owns row
+// r0 + t and keeps its 32 weights in registers.  H_gg is staged once per CTA
+// in shared memory as the upper triangle of H'_{ij} = H_ij + H_ji (j > i),
+// H'_ii = H_ii (528 floats, read as broadcast float4), so that
+// E = sum_i e_i * (sum_{j >= i} H'_ij e_j): 528 + 32 FMA per candidate.
+// Each thread evaluates two candidates per pass so every shared-memory load
+// feeds two FMAs.
+//
+// Exactness: the codes are exact (rint of the IEEE quotient w / Delta_k; the
+// quotient is formed as w * (1/Delta_k) and the IEEE division is redone for
+// the group whenever that product lands within 2^-18 of a rounding boundary,
+// which a 3-ulp error analysis shows is the only place the two can differ).
+// E is screened in float32 together with a rigorous bound
+//     |E32 - E| <= 80 u kappa S^2,   S = sum_i |e_i| sqrt|H_ii|,  u = 2^-24,
+// kappa = max(1, max_{i != j} |H_ij| / sqrt|H_ii H_jj|)  (= 1 for a PSD H)
+// which covers the 33-term FMA chains and the rounding of H'.  Every candidate
+// whose interval [E32 - b, E32 + b] can still contain the minimum is
+// re-scored in float64 (the top four lower bounds are kept; if four or more
+// are undecided, all K candidates are re-scored), and the float64 minimum
+// wins, smallest k on ties.
+#pragma once
+
+#include <utility>
+
+#include "device_common.cuh"
+
+namespace qat4 {
+
+constexpr int kSearchThreads = 128;
+constexpr int kTri = 528;          // entries of the upper triangle of a 32x32 block
+constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23: x + M - M = rint(x) for |x| < 2^22
+constexpr float kTieWindow = 0.5f - 3.814697265625e-06f;  // 0.5 - 2^-18
+constexpr float kBoundC = 80.0f * 5.9604644775390625e-08f;  // 80 * 2^-24
+
+// Row / column of entry p of the row-major upper triangle (j >= i) of a 32x32 matrix.
+__host__ __device__ constexpr int tri_row(int p) {
+    int i = 0;
+    while (p >= 32 - i) { p -= 32 - i; ++i; }
+    return i;
+}
+__host__ __device__ constexpr int tri_col(int p) {
+    int i = 0;
+    while (p >= 32 - i) { p -= 32 - i; ++i; }
+    return i + p;
+}
+static_assert(tri_row(527) == 31 && tri_col(527) == 31 && tri_col(31) == 31 && tri_row(32) == 1, "tri");
+
+struct SearchSmem {
+    float4 h32[kTri / 4];   // H' upper triangle, float32
+    double h64[kTri];       // same, float64 (H_ij + H_ji exact)
+    float4 sqrt_diag[8];    // sqrt(|H_ii|), rounded up
+    float hfull[32][33];    // staging copy of H_gg (padded)
+    unsigned kappa_bits;    // kappa as float bits (non-negative: int order == float order)
+};
+
+// e_i = fl(w_i - fl(dk * q_i)), q_i = clamp(rint(fl(w_i / dk)), -8, 7).
+__device__ __forceinline__ void group_error(const float (&w)[32], float dk, float (&e)[32]) {
+    const float rc = __frcp_rn(dk);
+    bool slow = !(fabsf(rc) <= 3.4028234663852886e38f);   // dk == 0 or 1/dk overflows
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const float r = fminf(fmaxf(__fmul_rn(w[i], rc), kQmin), kQmax);
+        const float q = __fsub_rn(__fadd_rn(r, kMagic), kMagic);
+        slow |= !(fabsf(__fsub_rn(r, q)) <= kTieWindow);
+        e[i] = __fsub_rn(w[i], __fmul_rn(dk, q));
+    }
+    if (slow) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float q = code_of(scaled_exact(w[i], dk));
+            e[i] = __fsub_rn(w[i], __fmul_rn(dk, q));
+        }
+    }
+}
+
+template <int P>
+__device__ __forceinline__ void tri_fma2(float h, const float (&e0)[32], const float (&e1)[32],
+                                         float& t0, float& t1, float& E0, float& E1) {
+    constexpr int i = tri_row(P);
+    constexpr int j = tri_col(P);
+    t0 = fmaf(h, e0[j], t0);
+    t1 = fmaf(h, e1[j], t1);
+    if constexpr (j == 31) {
+        E0 = fmaf(e0[i], t0, E0);
+        E1 = fmaf(e1[i], t1, E1);
+        t0 = 0.0f;
+        t1 = 0.0f;
+    }
+}
+
+template <int Q4>
+__device__ __forceinline__ void tri_quad2(const float4* h32, const float (&e0)[32], const float (&e1)[32],
+                                          float& t0, float& t1, float& E0, float& E1) {
+    const float4 h = h32[Q4];
+    tri_fma2<4 * Q4 + 0>(h.x, e0, e1, t0, t1, E0, E1);
+    tri_fma2<4 * Q4 + 1>(h.y, e0, e1, t0, t1, E0, E1);
+    tri_fma2<4 * Q4 + 2>(h.z, e0, e1, t0, t1, E0, E1);
+    tri_fma2<4 * Q4 + 3>(h.w, e0, e1, t0, t1, E0, E1);
+}
+
+template <int... Q4s>
+__device__ __forceinline__ void quad_form2_impl(std::integer_sequence<int, Q4s...>, const float4* h32,
+                                                const float (&e0)[32], const float (&e1)[32],
+                                                float& E0, float& E1) {
+    float t0 = 0.0f, t1 = 0.0f;
+    E0 = 0.0f;
+    E1 = 0.0f;
+    (tri_quad2<Q4s>(h32, e0, e1, t0, t1, E0, E1), ...);
+}
+
+// float32 screening values of two candidates.
+__device__ __forceinline__ void quad_form2(const float4* h32, const float (&e0)[32], const float (&e1)[32],
+                                           float& E0, float& E1) {
+    quad_form2_impl(std::make_integer_sequence<int, kTri / 4>{}, h32, e0, e1, E0, E1);
+}
+
+// float64 value of one candidate (the re-score).
+__device__ __forceinline__ double quad_form64(const double* h64, const float (&e)[32]) {
+    double ed[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ed[i] = static_cast<double>(e[i]);
+    double E = 0.0;
+    int p = 0;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        double t = 0.0;
+#pragma unroll
+        for (int j = i; j < 32; ++j) t = fma(h64[p++], ed[j], t);
+        E = fma(ed[i], t, E);
+    }
+    return E;
+}
+
+struct TopK4 {
+    float L[4];
+    int k[4];
+    __device__ __forceinline__ void init() {
+#pragma unroll
+        for (int a = 0; a < 4; ++a) { L[a] = __int_as_float(0x7f800000); k[a] = -1; }
+    }
+    // keeps the four smallest lower bounds, ascending
+    __device__ __forceinline__ void insert(float l, int kk) {
+        if (!(l < L[3])) return;
+        if (l < L[2]) {
+            L[3] = L[2]; k[3] = k[2];
+            if (l < L[1]) {
+                L[2] = L[1]; k[2] = k[1];
+                if (l < L[0]) { L[1] = L[0]; k[1] = k[0]; L[0] = l; k[0] = kk; }
+                else { L[1] = l; k[1] = kk; }
+            } else { L[2] = l; k[2] = kk; }
+        } else { L[3] = l; k[3] = kk; }
+    }
+};
+
+__global__ void __launch_bounds__(kSearchThreads, 3)
+scale_search_kernel(const float* __restrict__ W, int R, int C,
+                    const float* __restrict__ H, int64_t ldh,
+                    const float* __restrict__ alpha, int K,
+                    float* __restrict__ delta_out, int* __restrict__ idx_out,
+                    float* __restrict__ err_out) {
+    __shared__ __align__(16) SearchSmem sm;
+    const int g = blockIdx.y;
+    const int G = C / kGroup;
+    const int tid = threadIdx.x;
+
+    // ---- stage H_gg and its derived tables
+    const float* Hg = H + static_cast<int64_t>(g) * kGroup * ldh + static_cast<int64_t>(g) * kGroup;
+    for (int x = tid; x < 32 * 32; x += kSearchThreads) {
+        const int i = x >> 5, j = x & 31;
+        sm.hfull[i][j] = Hg[static_cast<int64_t>(i) * ldh + j];
+    }
+    if (tid == 0) sm.kappa_bits = __float_as_uint(1.0f);
+    __syncthreads();
+    float* h32f = reinterpret_cast<float*>(sm.h32);
+    float kap = 0.0f;
+    for (int p = tid; p < kTri; p += kSearchThreads) {
+        const int i = tri_row(p), j = tri_col(p);
+        const float a = sm.hfull[i][j], b = sm.hfull[j][i];
+        if (i == j) {
+            h32f[p] = a;
+            sm.h64[p] = static_cast<double>(a);
+        } else {
+            h32f[p] = __fadd_rn(a, b);
+            sm.h64[p] = static_cast<double>(a) + static_cast<double>(b);
+            const double m = fmax(fabs(static_cast<double>(a)), fabs(static_cast<double>(b)));
+            if (m != 0.0) {
+                const double den = sqrt(fabs(static_cast<double>(sm.hfull[i][i])) *
+                                        fabs(static_cast<double>(sm.hfull[j][j])));
+                const double ratio = den > 0.0 ? m / den : 1e300;
+                kap = fmaxf(kap, ratio > 3.0e38 ? __int_as_float(0x7f800000)
+                                                : __double2float_ru(ratio));
+            }
+        }
+    }
+    if (tid < 32) reinterpret_cast<float*>(sm.sqrt_diag)[tid] = __fsqrt_ru(fabsf(sm.hfull[tid][tid]));
+    atomicMax(&sm.kappa_bits, __float_as_uint(kap));
+    __syncthreads();
+
+    const int r = blockIdx.x * kSearchThreads + tid;
+    if (r >= R) return;
+    const float kappa = __uint_as_float(sm.kappa_bits);
+    const float bound_c = kBoundC * kappa;
+
+    float w[32];
+    const float4* wp = reinterpret_cast<const float4*>(W + static_cast<int64_t>(r) * C + g * kGroup);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) {
+        const float4 x = __ldg(wp + v);
+        w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+    }
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(w[i]));
+    const int64_t out = static_cast<int64_t>(r) * G + g;
+    if (m == 0.0f) {   // all-zero group: every candidate has zero error
+        delta_out[out] = 0.0f;
+        idx_out[out] = 0;
+        if (err_out) err_out[out] = 0.0f;
+        return;
+    }
+    const float base = __fdiv_rn(m, 7.0f);
+
+    TopK4 top;
+    top.init();
+    float upper = __int_as_float(0x7f800000);
+    for (int k = 0; k < K; k += 2) {
+        const int k1 = (k + 1 < K) ? k + 1 : k;
+        const float d0 = __fmul_rn(__ldg(alpha + k), base);
+        const float d1 = __fmul_rn(__ldg(alpha + k1), base);
+        float e0[32], e1[32];
+        group_error(w, d0, e0);
+        group_error(w, d1, e1);
+        float E0, E1;
+        quad_form2(sm.h32, e0, e1, E0, E1);
+        float S0 = 0.0f, S1 = 0.0f;
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            const float4 s4 = sm.sqrt_diag[v];
+            S0 = fmaf(fabsf(e0[4 * v + 0]), s4.x, S0);
+            S1 = fmaf(fabsf(e1[4 * v + 0]), s4.x, S1);
+            S0 = fmaf(fabsf(e0[4 * v + 1]), s4.y, S0);
+            S1 = fmaf(fabsf(e1[4 * v + 1]), s4.y, S1);
+            S0 = fmaf(fabsf(e0[4 * v + 2]), s4.z, S0);
+            S1 = fmaf(fabsf(e1[4 * v + 2]), s4.z, S1);
+            S0 = fmaf(fabsf(e0[4 * v + 3]), s4.w, S0);
+            S1 = fmaf(fabsf(e1[4 * v + 3]), s4.w, S1);
+        }
+        const float b0 = bound_c * S0 * S0;
+        const float b1 = bound_c * S1 * S1;
+        upper = fminf(upper, E0 + b0);
+        top.insert(E0 - b0, k);
+        if (k1 != k) {
+            upper = fminf(upper, E1 + b1);
+            top.insert(E1 - b1, k1);
+        }
+    }
+
+    // ---- float64 re-score of every candidate the screening could not exclude
+    int nfin = 0;
+#pragma unroll
+    for (int a = 0; a < 4; ++a) nfin += (top.k[a] >= 0 && top.L[a] <= upper) ? 1 : 0;
+    const bool overflow = (nfin == 4 && K > 4) || nfin == 0;
+    double best = 0.0;
+    int best_k = -1;
+    const int count = overflow ? K : nfin;
+    for (int a = 0; a < count; ++a) {
+        const int kk = overflow ? a : (a == 0 ? top.k[0] : a == 1 ? top.k[1] : a == 2 ? top.k[2] : top.k[3]);
+        float e[32];
+        group_error(w, __fmul_rn(__ldg(alpha + kk), base), e);
+        const double E = quad_form64(sm.h64, e);
+        if (best_k < 0 || E < best || (E == best && kk < best_k)) { best = E; best_k = kk; }
+    }
+    delta_out[out] = __fmul_rn(__ldg(alpha + best_k), base);
+    idx_out[out] = best_k;
+    if (err_out) err_out[out] = static_cast<float>(best);
+}
+
+}  // namespace qat4

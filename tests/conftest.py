@@ -18,3 +18,37 @@ def oracle_mod():
     import oracle
     oracle.lib()
     return oracle
+
+
+def gpu_available():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
+
+
+def pytest_collection_modifyitems(config, items):
+    if gpu_available():
+        return
+    skip = pytest.mark.skip(reason="no CUDA GPU on this host")
+    for item in items:
+        if "gpu" in item.keywords:
+            item.add_marker(skip)
+
+
+class _Cache:
+    """Session cache of generated workloads (inputs only; never kernel outputs)."""
+
+    def __init__(self):
+        self.store = {}
+
+    def get(self, key, make):
+        if key not in self.store:
+            self.store[key] = make()
+        return self.store[key]
+
+
+@pytest.fixture(scope="session")
+def cache():
+    return _Cache()

@@ -1,0 +1,85 @@
+"""The C ABI without a GPU: the library loads, exports every declared entry
+point, and rejects bad arguments on the host before anything is launched."""
+import ctypes as ct
+import os
+import re
+
+import numpy as np
+import pytest
+
+import int4_group_wise_b200 as q4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qat4.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qat4_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported_and_bound():
+    L = q4.lib()
+    names = _declared()
+    assert "qat4_hessian" in names and "qat4_scale_search" in names and len(names) >= 11
+    for n in names:
+        assert hasattr(L, n), n
+    assert sorted(q4.EXPORTS) == names
+    assert L.qat4_abi_version() == 1
+
+
+def test_status_strings():
+    for code, name in q4.STATUS.items():
+        assert q4.status_string(code).startswith(name)
+    assert "UNKNOWN" in q4.status_string(99)
+
+
+def test_grad_scale_constant():
+    assert q4.GRAD_SCALE == float(np.float32(1.0 / np.sqrt(224.0)))
+
+
+# Fake, 16-byte aligned non-null "device" addresses: validation rejects the
+# call before any pointer is dereferenced or any CUDA call is made.
+A = ct.c_void_p(0x10000)
+B = ct.c_void_p(0x20000)
+MIS = ct.c_void_p(0x20004)
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, 8, 64, A, A), 1),
+    ((A, 8, 64, None, A), 1),
+    ((A, 0, 64, A, A), 2),
+    ((A, 8, 48, A, A), 2),
+    ((A, 8, 0, A, A), 2),
+    ((MIS, 8, 64, A, A), 3),
+    ((A, 8, 64, A, MIS), 3),
+])
+def test_lsq_fwd_validation(args, code):
+    W, R, C, d, Q = args
+    assert q4.lib().qat4_lsq_fwd(W, d, R, C, Q, None) == code
+
+
+def test_lsq_bwd_and_fused_validation():
+    L = q4.lib()
+    assert L.qat4_lsq_bwd(A, A, None, 0, 4, 64, ct.c_float(1.0), A, A, None) == 1
+    assert L.qat4_lsq_bwd(A, A, A, 7, 4, 64, ct.c_float(1.0), A, A, None) == 4
+    assert L.qat4_lsq_bwd(A, A, MIS, 1, 4, 64, ct.c_float(1.0), A, A, None) == 3
+    assert L.qat4_lsq_fwd_bwd(A, A, A, 1, 4, 64, ct.c_float(1.0), None, A, A, None) == 1
+    assert L.qat4_lsq_fwd_bwd(A, A, A, 1, 4, 33, ct.c_float(1.0), A, A, A, None) == 2
+
+
+def test_pack_search_hessian_validation():
+    L = q4.lib()
+    assert L.qat4_pack_w4a16(A, A, 4, 64, None, A, None) == 1
+    assert L.qat4_pack_w4a16(A, A, -1, 64, A, A, None) == 2
+    assert L.qat4_pack_w4a16(A, A, 4, 64, A, MIS, None) == 3
+    assert L.qat4_scale_search(A, 4, 64, A, 64, A, 0, A, A, None, None) == 2      # K = 0
+    assert L.qat4_scale_search(A, 4, 64, A, 32, A, 5, A, A, None, None) == 2      # ldh < C
+    assert L.qat4_scale_search(A, 4, 64, A, 66, A, 5, A, A, None, None) == 3      # ldh not 16-B multiple
+    assert L.qat4_scale_search(A, 4, 64, A, 64, None, 5, A, A, None, None) == 1
+    assert L.qat4_hessian(None, 64, 64, A, None, 0, None) == 1
+    assert L.qat4_hessian(A, 0, 64, A, None, 0, None) == 2
+    assert L.qat4_hessian(A, 64, 40, A, None, 0, None) == 2
+    assert L.qat4_hessian(MIS, 64, 64, A, None, 0, None) == 3
+    assert L.qat4_selftest_bounded_wait(0, None) == 2
