@@ -108,18 +108,19 @@ int qat4_abi_version(void) { return 1; }
 
 // ------------------------------------------------------------------ Hessian
 size_t qat4_hessian_workspace_bytes(int64_t n, int64_t C) {
-    (void)n;
-    (void)C;
-    return 0;   // one CTA per output tile: no split-reduction scratch
+    if (n < 1 || C < 32 || C % 32 != 0 || C > 65536) return 0;
+    const qat4::HessPlan plan = qat4::hess_plan(n, C);
+    if (plan.split <= 1) return 0;
+    return static_cast<size_t>(plan.tiles) * plan.split * qat4::kPTile * qat4::kPTile * sizeof(float);
 }
 
 qat4_status qat4_hessian(const uint16_t* X, int64_t n, int64_t C, float* H,
                          void* workspace, size_t workspace_bytes, cudaStream_t stream) {
     if (!X || !H) return QAT4_ERR_NULL;
     if (n < 1 || n > (int64_t(1) << 31) - 1 || C < 32 || C % 32 != 0 || C > 65536) return QAT4_ERR_SHAPE;
-    if (!aligned16(X) || !aligned16(H)) return QAT4_ERR_ALIGN;
-    if (workspace_bytes < qat4_hessian_workspace_bytes(n, C)) return QAT4_ERR_WORKSPACE;
-    (void)workspace;
+    if (!aligned16(X) || !aligned16(H) || (workspace && !aligned16(workspace))) return QAT4_ERR_ALIGN;
+    const size_t need = qat4_hessian_workspace_bytes(n, C);
+    if (workspace_bytes < need || (need > 0 && !workspace)) return QAT4_ERR_WORKSPACE;
 
     int dev;
     DeviceInfo* info;
@@ -127,8 +128,8 @@ qat4_status qat4_hessian(const uint16_t* X, int64_t n, int64_t C, float* H,
     {
         std::lock_guard<std::mutex> lock(g_mutex);
         if (!info->hessian_attr) {
-            if (cudaFuncSetAttribute(qat4::hessian_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(qat4::kHSmemBytes)) != cudaSuccess)
+            if (cudaFuncSetAttribute(qat4::hessian_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(qat4::kPSmemBytes)) != cudaSuccess)
                 return QAT4_ERR_CUDA;
             info->hessian_attr = true;
         }
@@ -139,7 +140,7 @@ qat4_status qat4_hessian(const uint16_t* X, int64_t n, int64_t C, float* H,
     CUtensorMap tmap;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(n)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(C) * 2};
-    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(qat4::kHBK)};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(qat4::kPBK)};
     const cuuint32_t estr[2] = {1, 1};
     if (encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -149,14 +150,19 @@ qat4_status qat4_hessian(const uint16_t* X, int64_t n, int64_t C, float* H,
     qat4::HessParams p;
     p.n = n;
     p.C = static_cast<int>(C);
-    p.nb = static_cast<int>((C + qat4::kHBM - 1) / qat4::kHBM);
-    p.kblocks = static_cast<int>((n + qat4::kHBK - 1) / qat4::kHBK);
+    p.plan = qat4::hess_plan(n, C);
     p.inv_n = static_cast<float>(1.0 / static_cast<double>(n));
-    // generous bound: 4 s plus 100 ns per calibration row (a tile's mainloop
-    // takes ~2 ns per row at full rate)
+    // generous bound: 4 s plus 100 ns per calibration row (a chunk of the
+    // mainloop takes ~2 ns per row at full rate)
     p.limit_ns = 4000000000ull + 100ull * static_cast<uint64_t>(n);
-    const unsigned tiles = static_cast<unsigned>(p.nb) * (p.nb + 1) / 2;
-    qat4::hessian_tc_kernel<<<tiles, qat4::kHThreads, qat4::kHSmemBytes, stream>>>(tmap, p, H);
+    const unsigned ctas = 2u * static_cast<unsigned>(p.plan.tiles) * static_cast<unsigned>(p.plan.split);
+    qat4::hessian_pair_kernel<<<ctas, qat4::kPThreads, qat4::kPSmemBytes, stream>>>(
+        tmap, p, H, static_cast<float*>(workspace));
+    if (cudaGetLastError() != cudaSuccess) return QAT4_ERR_CUDA;
+    if (p.plan.split > 1) {
+        const dim3 grid(static_cast<unsigned>(p.plan.tiles), 64);
+        qat4::hessian_reduce_kernel<<<grid, 256, 0, stream>>>(static_cast<const float*>(workspace), p, H);
+    }
     return launch_status();
 }
 

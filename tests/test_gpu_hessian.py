@@ -83,6 +83,46 @@ def test_hessian_full_size_sampled(cfg, cache, oracle_mod):
     assert (num / den) ** 0.5 <= 1e-3, (num / den) ** 0.5
 
 
+@pytest.mark.parametrize("n,C", [(40000, 3072), (50000, 2048), (20000, 512)])
+def test_hessian_multi_chunk_ragged(n, C, oracle_mod):
+    """n spans several 16384-row promotion chunks with a ragged last chunk and a ragged last
+    64-row stage; (40000, 3072) stores H directly, the others split n and reduce partials."""
+    Xb = inputs.activations(n, C, seed=n, cfg=62, name="X", outliers=C // 100)
+    X, H = _gpu_h(Xb)
+    Hg = H.cpu().numpy()
+    np.testing.assert_array_equal(Hg, Hg.T)
+    rng = np.random.default_rng(n)
+    num = den = 0.0
+    blocks = [(0, 0), (C - 128, C - 128)] + [tuple(int(v) * 64 for v in rng.integers(0, C // 64 - 1, 2))
+                                             for _ in range(3)]
+    for r0, c0 in blocks:
+        ref = oracle_mod.hessian_block(Xb, r0, 128 if r0 + 128 <= C else 64, c0, 128 if c0 + 128 <= C else 64)
+        got = Hg[r0:r0 + ref.shape[0], c0:c0 + ref.shape[1]]
+        num += float(np.sum((got - ref) ** 2))
+        den += float(np.sum(ref ** 2))
+    assert (num / den) ** 0.5 <= 1e-3, (num / den) ** 0.5
+
+
+def test_hessian_workspace_contract():
+    """The call rejects a missing or short workspace when n is split, and ignores it otherwise."""
+    Xb = inputs.activations(4096, 512, seed=5, cfg=63, name="X")
+    X = torch.from_numpy(Xb.view(np.int16)).cuda().view(torch.bfloat16)
+    need = q4.hessian_workspace_bytes(4096, 512)
+    assert need > 0
+    H = torch.empty((512, 512), dtype=torch.float32, device="cuda")
+    L = q4.lib()
+    st = torch.cuda.current_stream().cuda_stream
+    import ctypes as ct
+    assert L.qat4_hessian(ct.c_void_p(X.data_ptr()), 4096, 512, ct.c_void_p(H.data_ptr()), None, 0,
+                          ct.c_void_p(st)) == 5
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    assert L.qat4_hessian(ct.c_void_p(X.data_ptr()), 4096, 512, ct.c_void_p(H.data_ptr()),
+                          ct.c_void_p(ws.data_ptr()), need - 16, ct.c_void_p(st)) == 5
+    assert L.qat4_hessian(ct.c_void_p(X.data_ptr()), 4096, 512, ct.c_void_p(H.data_ptr()),
+                          ct.c_void_p(ws.data_ptr()), need, ct.c_void_p(st)) == 0
+    q4.sync_check()
+
+
 def test_bounded_wait_reports_timeout_and_context_survives():
     assert q4.selftest_bounded_wait(20_000_000) == 7      # QAT4_ERR_TIMEOUT after ~20 ms
     q4.sync_check()                                        # cleared
