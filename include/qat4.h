@@ -164,6 +164,30 @@ qat4_status qat4_lsq_fwd_bwd(const float *W, const float *delta, const void *G, 
 qat4_status qat4_pack_w4a16(const float *W, const float *delta, int64_t R, int64_t C,
                             uint8_t *packed, uint16_t *scales, cudaStream_t stream);
 
+/* Same result as qat4_hessian, for callers that cannot allocate device memory
+ * themselves -- for example code running inside an engine or framework that
+ * owns all device memory through its own allocator or a fixed budget, or a
+ * latency-critical loop where cudaMalloc/cudaFree (which may synchronise the
+ * device) are not acceptable.  The pages describe no such variant; it has no
+ * counterpart there.
+ *
+ *  X, n, C, H  as for qat4_hessian.  No workspace argument: the scratch is a
+ *              static device array of 19,398,656 bytes (18.5 MiB) inside the
+ *              library, which every GPU that loads the library holds until the
+ *              process exits.  It covers every (n, C) the planner accepts;
+ *              a shape that needed more would be rejected with
+ *              QAT4_ERR_WORKSPACE.
+ *  The call allocates nothing: no cudaMalloc, cudaFree or allocating library
+ *  routine.  Its first call on a device (with that device current) looks up
+ *  the array's device address once; make that first call before any stream
+ *  capture.  All calls on a device share the one array: two calls whose
+ *  kernels overlap on the GPU (different streams, or other host threads)
+ *  race on it and must be ordered by the caller.  Every byte of the scratch
+ *  that is read is first written by the same call, so nothing from the
+ *  previous call leaks into the result.
+ *  Errors: QAT4_ERR_NULL, _SHAPE, _ALIGN, _WORKSPACE, _CUDA. */
+qat4_status qat4_hessian_noalloc(const uint16_t *X, int64_t n, int64_t C, float *H, cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the library's device error
  * word for the current device.  Returns QAT4_ERR_TIMEOUT if a kernel gave up
  * a bounded wait since the last check, QAT4_ERR_CUDA if synchronisation

@@ -7,7 +7,7 @@ device pointers plus the current CUDA stream to the C ABI in
 ``libqat4.so``; if that library is missing, every call raises.
 
 Functions (same names as the C entry points, without the ``qat4_`` prefix):
-``hessian``, ``hessian_workspace_bytes``, ``scale_search``, ``lsq_fwd``,
+``hessian``, ``hessian_workspace_bytes``, ``hessian_noalloc``, ``scale_search``, ``lsq_fwd``,
 ``lsq_bwd``, ``lsq_fwd_bwd``, ``pack_w4a16``, ``sync_check``,
 ``status_string``, ``selftest_bounded_wait``.
 """
@@ -34,6 +34,7 @@ EXPORTS = {
     "qat4_abi_version": (ct.c_int, []),
     "qat4_hessian_workspace_bytes": (_Z, [_I64, _I64]),
     "qat4_hessian": (ct.c_int, [_P, _I64, _I64, _P, _P, _Z, _P]),
+    "qat4_hessian_noalloc": (ct.c_int, [_P, _I64, _I64, _P, _P]),
     "qat4_scale_search": (ct.c_int, [_P, _I64, _I64, _P, _I64, _P, _I32, _P, _P, _P, _P]),
     "qat4_lsq_fwd": (ct.c_int, [_P, _P, _I64, _I64, _P, _P]),
     "qat4_lsq_bwd": (ct.c_int, [_P, _P, _P, ct.c_int, _I64, _I64, _F, _P, _P, _P]),
@@ -122,6 +123,21 @@ def hessian(X, H=None, workspace=None, stream=None):
     wp = _dev(workspace, "workspace", torch.uint8) if workspace is not None else None
     wbytes = workspace.numel() if workspace is not None else 0
     _check(L.qat4_hessian(_dev(X, "X"), n, C, _dev(H, "H"), wp, wbytes, _stream(stream)), "qat4_hessian")
+    return H
+
+
+def hessian_noalloc(X, H=None, stream=None):
+    """H = X^T X / n using the library's built-in scratch instead of a caller workspace.
+
+    For callers that must not allocate device memory on their own (H may be
+    passed in preallocated).  Calls that overlap on the GPU share the scratch
+    and race; see include/qat4.h."""
+    import torch
+    L = lib()
+    _dev(X, "X", torch.bfloat16)
+    n, C = X.shape
+    H = _out(H, "H", (C, C), torch.float32, X)
+    _check(L.qat4_hessian_noalloc(_dev(X, "X"), n, C, _dev(H, "H"), _stream(stream)), "qat4_hessian_noalloc")
     return H
 
 

@@ -289,3 +289,50 @@ extern "C" qat4_status qat4_selftest_bounded_wait(int64_t limit_ns, cudaStream_t
     qat4::bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(limit_ns));
     return launch_status();
 }
+
+// ------------------------------------------------------ no-allocation variant
+// Some callers of this library cannot allocate device memory themselves: code
+// that runs inside an engine or framework which owns every byte of device
+// memory (a caching allocator or a fixed memory budget that a stray cudaMalloc
+// would break), and latency-critical loops in which cudaMalloc/cudaFree, which
+// may synchronise the device, are not acceptable.  qat4_hessian_noalloc serves
+// them: its scratch is the file-scope array below, which every GPU that loads
+// this library holds until the process exits.
+namespace {
+
+// Largest workspace the Hessian planner can ask for: n is split only while
+// tiles * S <= 74, and each (tile, part) unit needs one 256 x 256 fp32 partial.
+constexpr size_t kNoallocScratchBytes =
+    static_cast<size_t>(qat4::kPPairsPerGpu) * qat4::kPTile * qat4::kPTile * sizeof(float);  // 18.5 MiB
+
+static __device__ __align__(256) unsigned char g_hessian_scratch[kNoallocScratchBytes];
+
+void* g_scratch_addr[kMaxDevices] = {};   // device address of g_hessian_scratch, per device
+
+}  // namespace
+
+extern "C" qat4_status qat4_hessian_noalloc(const uint16_t* X, int64_t n, int64_t C, float* H,
+                                            cudaStream_t stream) {
+    if (!X || !H) return QAT4_ERR_NULL;
+    if (n < 1 || n > (int64_t(1) << 31) - 1 || C < 32 || C % 32 != 0 || C > 65536) return QAT4_ERR_SHAPE;
+    const size_t need = qat4_hessian_workspace_bytes(n, C);
+    if (need > kNoallocScratchBytes) return QAT4_ERR_WORKSPACE;   // larger than the built-in scratch
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QAT4_ERR_CUDA;
+    void* scratch = nullptr;
+    {
+        // One-time set-up per device, with that device current: host code only
+        // knows a stand-in for the array, so its device address is looked up.
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (g_scratch_addr[dev] == nullptr) {
+            void* addr = nullptr;
+            if (cudaGetSymbolAddress(&addr, g_hessian_scratch) != cudaSuccess || addr == nullptr)
+                return QAT4_ERR_CUDA;
+            g_scratch_addr[dev] = addr;
+        }
+        scratch = g_scratch_addr[dev];
+    }
+    // The kernels overwrite every scratch byte they later read, so the previous
+    // call's contents need no clearing.
+    return qat4_hessian(X, n, C, H, scratch, kNoallocScratchBytes, stream);
+}
