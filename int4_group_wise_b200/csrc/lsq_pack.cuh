@@ -52,8 +52,8 @@ __device__ __forceinline__ LsqElem lsq_elem(float w, float d, float g) {
     return o;
 }
 
-// FWD: write Q.  BWD: write grad_W and grad_delta.
-template <typename GT, bool FWD, bool BWD>
+// FWD: write Q.  BWD: write grad_W and grad_delta.  U steps in flight per warp.
+template <typename GT, bool FWD, bool BWD, int U = kUnroll>
 __global__ void __launch_bounds__(kStreamThreads)
 lsq_kernel(const float* __restrict__ W, const float* __restrict__ delta,
            const GT* __restrict__ G, int64_t nquads, float grad_scale,
@@ -65,12 +65,12 @@ lsq_kernel(const float* __restrict__ W, const float* __restrict__ delta,
     const int64_t nsteps_ceil = (nquads + 31) >> 5;
     (void)nsteps;
 
-    for (int64_t s0 = warp * kUnroll; s0 < nsteps_ceil; s0 += nwarps * kUnroll) {
-        float4 w[kUnroll], g[kUnroll];
-        float d[kUnroll];
-        bool valid[kUnroll];
+    for (int64_t s0 = warp * U; s0 < nsteps_ceil; s0 += nwarps * U) {
+        float4 w[U], g[U];
+        float d[U];
+        bool valid[U];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int64_t quad = (s0 + u) * 32 + lane;
             valid[u] = quad < nquads;
             if (valid[u]) {
@@ -84,7 +84,7 @@ lsq_kernel(const float* __restrict__ W, const float* __restrict__ delta,
             }
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < U; ++u) {
             const int64_t quad = (s0 + u) * 32 + lane;
             const LsqElem e0 = lsq_elem(w[u].x, d[u], BWD ? g[u].x : 0.f);
             const LsqElem e1 = lsq_elem(w[u].y, d[u], BWD ? g[u].y : 0.f);
@@ -142,6 +142,7 @@ __device__ __forceinline__ uint32_t pack4(float4 w, float d) {
 // W4A16 export.  Lane l converts the float4 at elements 4l..4l+3 of a
 // 128-element step into two bytes (one coalesced 2-byte store); lanes 0, 8,
 // 16, 24 also write their group's binary16 scale.
+template <int U = 4>
 __global__ void __launch_bounds__(kStreamThreads)
 pack_w4a16_kernel(const float* __restrict__ W, const float* __restrict__ delta, int64_t nquads,
                   uint16_t* __restrict__ packed16, uint16_t* __restrict__ scales) {
@@ -149,7 +150,6 @@ pack_w4a16_kernel(const float* __restrict__ W, const float* __restrict__ delta, 
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kStreamThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kStreamThreads) >> 5;
     const int64_t nsteps_ceil = (nquads + 31) >> 5;
-    constexpr int U = 4;
     for (int64_t s0 = warp * U; s0 < nsteps_ceil; s0 += nwarps * U) {
         float4 w[U];
         float d[U];

@@ -32,6 +32,7 @@ bool valid_rc(int64_t R, int64_t C) {
 struct DeviceInfo {
     int sms = 0;
     bool hessian_attr = false;
+    bool search_attr = false;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mutex;
@@ -175,9 +176,21 @@ qat4_status qat4_scale_search(const float* W, int64_t R, int64_t C, const float*
     if (!aligned16(W) || !aligned16(H) || !aligned16(alpha) || !aligned16(delta) || !aligned16(idx) ||
         (best_err && !aligned16(best_err)) || (ldh % 4) != 0)
         return QAT4_ERR_ALIGN;
+    int dev;
+    DeviceInfo* info;
+    if (!device_info(&dev, &info)) return QAT4_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!info->search_attr) {
+            if (cudaFuncSetAttribute(qat4::scale_search_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(sizeof(qat4::SearchSmem))) != cudaSuccess)
+                return QAT4_ERR_CUDA;
+            info->search_attr = true;
+        }
+    }
     const dim3 grid(static_cast<unsigned>((R + qat4::kSearchThreads - 1) / qat4::kSearchThreads),
                     static_cast<unsigned>(C / 32));
-    qat4::scale_search_kernel<<<grid, qat4::kSearchThreads, 0, stream>>>(
+    qat4::scale_search_kernel<3><<<grid, qat4::kSearchThreads, sizeof(qat4::SearchSmem), stream>>>(
         W, static_cast<int>(R), static_cast<int>(C), H, ldh, alpha, K, delta, idx, best_err);
     return launch_status();
 }
@@ -249,7 +262,7 @@ qat4_status qat4_pack_w4a16(const float* W, const float* delta, int64_t R, int64
     DeviceInfo* info;
     if (!device_info(&dev, &info)) return QAT4_ERR_CUDA;
     const int64_t nquads = R * C / 4;
-    qat4::pack_w4a16_kernel<<<stream_blocks(nquads, info->sms, 4), qat4::kStreamThreads, 0, stream>>>(
+    qat4::pack_w4a16_kernel<4><<<stream_blocks(nquads, info->sms, 4), qat4::kStreamThreads, 0, stream>>>(
         W, delta, nquads, reinterpret_cast<uint16_t*>(packed), scales);
     return launch_status();
 }

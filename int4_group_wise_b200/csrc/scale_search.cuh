@@ -10,10 +10,11 @@
 // Mapping: one CTA = one column group g x 128 rows; thread t owns row
 // r0 + t and keeps its 32 weights in registers.  H_gg is staged once per CTA
 // in shared memory as the upper triangle of H'_{ij} = H_ij + H_ji (j > i),
-// H'_ii = H_ii (528 floats, read as broadcast float4), so that
-// E = sum_i e_i * (sum_{j >= i} H'_ij e_j): 528 + 32 FMA per candidate.
-// Each thread evaluates two candidates per pass so every shared-memory load
-// feeds two FMAs.
+// H'_ii = H_ii (528 floats, stored twice and read as broadcast float4), so
+// that E = sum_i e_i * (sum_{j >= i} H'_ij e_j): 528 + 32 FMA per candidate.
+// Each thread evaluates two candidates per pass with packed FP32x2
+// instructions (one FFMA2 = one FMA of each candidate); the quantization
+// steps are packed the same way.
 //
 // Exactness: the codes are exact (rint of the IEEE quotient w / Delta_k; the
 // quotient is formed as w * (1/Delta_k) and the IEEE division is redone for
@@ -29,6 +30,7 @@
 // wins, smallest k on ties.
 #pragma once
 
+#include <cstddef>
 #include <utility>
 
 #include "device_common.cuh"
@@ -54,16 +56,40 @@ __host__ __device__ constexpr int tri_col(int p) {
 }
 static_assert(tri_row(527) == 31 && tri_col(527) == 31 && tri_col(31) == 31 && tri_row(32) == 1, "tri");
 
+constexpr int kSlot = 36;          // floats per thread slot (144 B: float4-aligned, few bank conflicts)
+
 struct SearchSmem {
-    float4 h32[kTri / 4];   // H' upper triangle, float32
+    float4 h32[kTri / 2];   // H' upper triangle, float32, each entry twice: (h_p, h_p, h_p+1, h_p+1)
     double h64[kTri];       // same, float64 (H_ij + H_ji exact)
     float4 sqrt_diag[8];    // sqrt(|H_ii|), rounded up
     float hfull[32][33];    // staging copy of H_gg (padded)
     unsigned kappa_bits;    // kappa as float bits (non-negative: int order == float order)
+    // per-thread copies of the 32 weights and of an error vector, used only by
+    // the exact (IEEE division) path so that it stays out of the unrolled loop
+    alignas(16) float wslot[kSearchThreads * kSlot];
+    alignas(16) float eslot[kSearchThreads * kSlot];
 };
+// every float4 access below needs these offsets to be multiples of 16 bytes
+static_assert(sizeof(float4) * (kTri / 2) == 2 * kTri * sizeof(float) && offsetof(SearchSmem, h32) % 16 == 0 && offsetof(SearchSmem, sqrt_diag) % 16 == 0 &&
+              offsetof(SearchSmem, h64) % 8 == 0 && offsetof(SearchSmem, wslot) % 16 == 0 &&
+              offsetof(SearchSmem, eslot) % 16 == 0 && (kSlot * 4) % 16 == 0, "SearchSmem alignment");
+
+// Exact error vector of one candidate from the weights parked in shared
+// memory: q = clamp(rint(w / dk), -8, 7) with the IEEE division, in a rolled
+// loop (taken only near a rounding boundary or when 1/dk is not finite).
+__device__ __noinline__ void group_error_exact(const float* wslot, float dk, float* eslot) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i) {
+        const float wi = wslot[i];
+        const float q = code_of(scaled_exact(wi, dk));
+        eslot[i] = __fsub_rn(wi, __fmul_rn(dk, q));
+    }
+}
 
 // e_i = fl(w_i - fl(dk * q_i)), q_i = clamp(rint(fl(w_i / dk)), -8, 7).
-__device__ __forceinline__ void group_error(const float (&w)[32], float dk, float (&e)[32]) {
+// wslot / eslot: this thread's shared-memory slots (wslot holds w).
+__device__ __forceinline__ void group_error(const float (&w)[32], float dk, float (&e)[32],
+                                            const float* wslot, float* eslot) {
     const float rc = __frcp_rn(dk);
     bool slow = !(fabsf(rc) <= 3.4028234663852886e38f);   // dk == 0 or 1/dk overflows
 #pragma unroll
@@ -74,53 +100,84 @@ __device__ __forceinline__ void group_error(const float (&w)[32], float dk, floa
         e[i] = __fsub_rn(w[i], __fmul_rn(dk, q));
     }
     if (slow) {
+        group_error_exact(wslot, dk, eslot);
+        const float4* e4 = reinterpret_cast<const float4*>(eslot);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const float q = code_of(scaled_exact(w[i], dk));
-            e[i] = __fsub_rn(w[i], __fmul_rn(dk, q));
+        for (int v = 0; v < 8; ++v) {
+            const float4 x = e4[v];
+            e[4 * v] = x.x; e[4 * v + 1] = x.y; e[4 * v + 2] = x.z; e[4 * v + 3] = x.w;
         }
     }
 }
 
+// Two candidates at once: element j of the pair register holds (e0_j, e1_j);
+// one packed FMA (FFMA2) advances both candidates' row sums.
 template <int P>
-__device__ __forceinline__ void tri_fma2(float h, const float (&e0)[32], const float (&e1)[32],
-                                         float& t0, float& t1, float& E0, float& E1) {
+__device__ __forceinline__ void tri_ffma2(float2 h, const float2 (&e)[32], float2& t, float2& E) {
     constexpr int i = tri_row(P);
     constexpr int j = tri_col(P);
-    t0 = fmaf(h, e0[j], t0);
-    t1 = fmaf(h, e1[j], t1);
+    t = __ffma2_rn(h, e[j], t);
     if constexpr (j == 31) {
-        E0 = fmaf(e0[i], t0, E0);
-        E1 = fmaf(e1[i], t1, E1);
-        t0 = 0.0f;
-        t1 = 0.0f;
+        E = __ffma2_rn(e[i], t, E);
+        t = make_float2(0.0f, 0.0f);
     }
 }
 
-template <int Q4>
-__device__ __forceinline__ void tri_quad2(const float4* h32, const float (&e0)[32], const float (&e1)[32],
-                                          float& t0, float& t1, float& E0, float& E1) {
-    const float4 h = h32[Q4];
-    tri_fma2<4 * Q4 + 0>(h.x, e0, e1, t0, t1, E0, E1);
-    tri_fma2<4 * Q4 + 1>(h.y, e0, e1, t0, t1, E0, E1);
-    tri_fma2<4 * Q4 + 2>(h.z, e0, e1, t0, t1, E0, E1);
-    tri_fma2<4 * Q4 + 3>(h.w, e0, e1, t0, t1, E0, E1);
+template <int Q2>
+__device__ __forceinline__ void tri_pair2(const float4* h32, const float2 (&e)[32], float2& t, float2& E) {
+    const float4 h = h32[Q2];                     // (h_p, h_p, h_p+1, h_p+1)
+    tri_ffma2<2 * Q2 + 0>(make_float2(h.x, h.y), e, t, E);
+    tri_ffma2<2 * Q2 + 1>(make_float2(h.z, h.w), e, t, E);
 }
 
-template <int... Q4s>
-__device__ __forceinline__ void quad_form2_impl(std::integer_sequence<int, Q4s...>, const float4* h32,
-                                                const float (&e0)[32], const float (&e1)[32],
-                                                float& E0, float& E1) {
-    float t0 = 0.0f, t1 = 0.0f;
-    E0 = 0.0f;
-    E1 = 0.0f;
-    (tri_quad2<Q4s>(h32, e0, e1, t0, t1, E0, E1), ...);
+template <int... Q2s>
+__device__ __forceinline__ float2 quad_form_pair_impl(std::integer_sequence<int, Q2s...>, const float4* h32,
+                                                      const float2 (&e)[32]) {
+    float2 t = make_float2(0.0f, 0.0f), E = make_float2(0.0f, 0.0f);
+    (tri_pair2<Q2s>(h32, e, t, E), ...);
+    return E;
 }
 
-// float32 screening values of two candidates.
-__device__ __forceinline__ void quad_form2(const float4* h32, const float (&e0)[32], const float (&e1)[32],
-                                           float& E0, float& E1) {
-    quad_form2_impl(std::make_integer_sequence<int, kTri / 4>{}, h32, e0, e1, E0, E1);
+// float32 screening values of two candidates, E.x and E.y.
+__device__ __forceinline__ float2 quad_form_pair(const float4* h32, const float2 (&e)[32]) {
+    return quad_form_pair_impl(std::make_integer_sequence<int, kTri / 2>{}, h32, e);
+}
+
+// Error vectors of two candidates (dk.x, dk.y) in packed form; every
+// component goes through exactly the operations of group_error, so the
+// values are bit-identical to it.
+__device__ __forceinline__ void group_error_pair(const float2 (&w2)[32], float2 dk, float2 (&e)[32],
+                                                 const float* wslot, float* eslot) {
+    const float2 rc = make_float2(__frcp_rn(dk.x), __frcp_rn(dk.y));
+    bool slow = !(fabsf(rc.x) <= 3.4028234663852886e38f) || !(fabsf(rc.y) <= 3.4028234663852886e38f);
+    const float2 M = make_float2(kMagic, kMagic);
+    const float2 negM = make_float2(-kMagic, -kMagic);
+    const float2 neg1 = make_float2(-1.0f, -1.0f);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        float2 r = __fmul2_rn(w2[i], rc);
+        r.x = fminf(fmaxf(r.x, kQmin), kQmax);
+        r.y = fminf(fmaxf(r.y, kQmin), kQmax);
+        const float2 q = __fadd2_rn(__fadd2_rn(r, M), negM);     // rint, exact for |r| <= 8
+        const float2 f = __ffma2_rn(q, neg1, r);                  // r - q
+        slow |= !(fabsf(f.x) <= kTieWindow) || !(fabsf(f.y) <= kTieWindow);
+        e[i] = __ffma2_rn(__fmul2_rn(dk, q), neg1, w2[i]);       // w - fl(dk * q)
+    }
+    if (slow) {
+        const float4* e4 = reinterpret_cast<const float4*>(eslot);
+        group_error_exact(wslot, dk.x, eslot);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            const float4 x = e4[v];
+            e[4 * v].x = x.x; e[4 * v + 1].x = x.y; e[4 * v + 2].x = x.z; e[4 * v + 3].x = x.w;
+        }
+        group_error_exact(wslot, dk.y, eslot);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) {
+            const float4 x = e4[v];
+            e[4 * v].y = x.x; e[4 * v + 1].y = x.y; e[4 * v + 2].y = x.z; e[4 * v + 3].y = x.w;
+        }
+    }
 }
 
 // float64 value of one candidate (the re-score).
@@ -161,13 +218,15 @@ struct TopK4 {
     }
 };
 
-__global__ void __launch_bounds__(kSearchThreads, 3)
+template <int MINB>
+__global__ void __launch_bounds__(kSearchThreads, MINB)
 scale_search_kernel(const float* __restrict__ W, int R, int C,
                     const float* __restrict__ H, int64_t ldh,
                     const float* __restrict__ alpha, int K,
                     float* __restrict__ delta_out, int* __restrict__ idx_out,
                     float* __restrict__ err_out) {
-    __shared__ __align__(16) SearchSmem sm;
+    extern __shared__ __align__(16) uint8_t search_smem_raw[];
+    SearchSmem& sm = *reinterpret_cast<SearchSmem*>(search_smem_raw);
     const int g = blockIdx.y;
     const int G = C / kGroup;
     const int tid = threadIdx.x;
@@ -186,10 +245,13 @@ scale_search_kernel(const float* __restrict__ W, int R, int C,
         const int i = tri_row(p), j = tri_col(p);
         const float a = sm.hfull[i][j], b = sm.hfull[j][i];
         if (i == j) {
-            h32f[p] = a;
+            h32f[2 * p] = a;
+            h32f[2 * p + 1] = a;
             sm.h64[p] = static_cast<double>(a);
         } else {
-            h32f[p] = __fadd_rn(a, b);
+            const float hp = __fadd_rn(a, b);
+            h32f[2 * p] = hp;
+            h32f[2 * p + 1] = hp;
             sm.h64[p] = static_cast<double>(a) + static_cast<double>(b);
             const double m = fmax(fabs(static_cast<double>(a)), fabs(static_cast<double>(b)));
             if (m != 0.0) {
@@ -228,39 +290,46 @@ scale_search_kernel(const float* __restrict__ W, int R, int C,
         return;
     }
     const float base = __fdiv_rn(m, 7.0f);
+    float* wslot = sm.wslot + tid * kSlot;
+    float* eslot = sm.eslot + tid * kSlot;
+    {
+        float4* w4 = reinterpret_cast<float4*>(wslot);
+#pragma unroll
+        for (int v = 0; v < 8; ++v) w4[v] = make_float4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+    }
 
     TopK4 top;
     top.init();
     float upper = __int_as_float(0x7f800000);
+    float2 w2[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) w2[i] = make_float2(w[i], w[i]);
     for (int k = 0; k < K; k += 2) {
         const int k1 = (k + 1 < K) ? k + 1 : k;
-        const float d0 = __fmul_rn(__ldg(alpha + k), base);
-        const float d1 = __fmul_rn(__ldg(alpha + k1), base);
-        float e0[32], e1[32];
-        group_error(w, d0, e0);
-        group_error(w, d1, e1);
-        float E0, E1;
-        quad_form2(sm.h32, e0, e1, E0, E1);
+        const float2 dk = make_float2(__fmul_rn(__ldg(alpha + k), base), __fmul_rn(__ldg(alpha + k1), base));
+        float2 e[32];
+        group_error_pair(w2, dk, e, wslot, eslot);
+        const float2 E = quad_form_pair(sm.h32, e);
         float S0 = 0.0f, S1 = 0.0f;
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
             const float4 s4 = sm.sqrt_diag[v];
-            S0 = fmaf(fabsf(e0[4 * v + 0]), s4.x, S0);
-            S1 = fmaf(fabsf(e1[4 * v + 0]), s4.x, S1);
-            S0 = fmaf(fabsf(e0[4 * v + 1]), s4.y, S0);
-            S1 = fmaf(fabsf(e1[4 * v + 1]), s4.y, S1);
-            S0 = fmaf(fabsf(e0[4 * v + 2]), s4.z, S0);
-            S1 = fmaf(fabsf(e1[4 * v + 2]), s4.z, S1);
-            S0 = fmaf(fabsf(e0[4 * v + 3]), s4.w, S0);
-            S1 = fmaf(fabsf(e1[4 * v + 3]), s4.w, S1);
+            S0 = fmaf(fabsf(e[4 * v + 0].x), s4.x, S0);
+            S1 = fmaf(fabsf(e[4 * v + 0].y), s4.x, S1);
+            S0 = fmaf(fabsf(e[4 * v + 1].x), s4.y, S0);
+            S1 = fmaf(fabsf(e[4 * v + 1].y), s4.y, S1);
+            S0 = fmaf(fabsf(e[4 * v + 2].x), s4.z, S0);
+            S1 = fmaf(fabsf(e[4 * v + 2].y), s4.z, S1);
+            S0 = fmaf(fabsf(e[4 * v + 3].x), s4.w, S0);
+            S1 = fmaf(fabsf(e[4 * v + 3].y), s4.w, S1);
         }
         const float b0 = bound_c * S0 * S0;
-        const float b1 = bound_c * S1 * S1;
-        upper = fminf(upper, E0 + b0);
-        top.insert(E0 - b0, k);
+        upper = fminf(upper, E.x + b0);
+        top.insert(E.x - b0, k);
         if (k1 != k) {
-            upper = fminf(upper, E1 + b1);
-            top.insert(E1 - b1, k1);
+            const float b1 = bound_c * S1 * S1;
+            upper = fminf(upper, E.y + b1);
+            top.insert(E.y - b1, k1);
         }
     }
 
@@ -275,7 +344,7 @@ scale_search_kernel(const float* __restrict__ W, int R, int C,
     for (int a = 0; a < count; ++a) {
         const int kk = overflow ? a : (a == 0 ? top.k[0] : a == 1 ? top.k[1] : a == 2 ? top.k[2] : top.k[3]);
         float e[32];
-        group_error(w, __fmul_rn(__ldg(alpha + kk), base), e);
+        group_error(w, __fmul_rn(__ldg(alpha + kk), base), e, wslot, eslot);
         const double E = quad_form64(sm.h64, e);
         if (best_k < 0 || E < best || (E == best && kk < best_k)) { best = E; best_k = kk; }
     }

@@ -70,6 +70,21 @@ def test_search_identity_and_ongrid(oracle_mod):
     assert torch.all(i == 100) and torch.all(e == 0) and torch.all(d == f32(2.0 ** -7))
 
 
+def test_search_exact_division_path(oracle_mod):
+    """Weights at exact half-integer multiples of a power-of-two step land on rounding ties at
+    alpha = 1 (the exact-division path), and alpha = 0 gives Delta = 0 (1/Delta not finite)."""
+    rng = np.random.default_rng(11)
+    R, C = 70, 96
+    step = f32(2.0 ** -7)
+    q = rng.integers(-7, 7, size=(R, C)).astype(f32) + f32(0.5)
+    q[:, ::32] = 7.0                                   # max |w| = 7 steps: base = step exactly
+    W = (step * q).astype(f32)
+    X, Xb = None, inputs.activations(128, C, seed=3, cfg=51, name="X")
+    H = oracle_mod.hessian(Xb).astype(f32)
+    alpha = np.array([0.0, 0.5, 0.75, 1.0, 1.25], f32)
+    check_search(W, H, alpha, oracle_mod)
+
+
 def test_search_non_psd_and_padded_ldh(oracle_mod):
     """A symmetric indefinite H (kappa > 1) and a row stride larger than C."""
     rng = np.random.default_rng(10)
