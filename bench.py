@@ -51,6 +51,41 @@ CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.a
 
 
 # --------------------------------------------------------------------------- setup
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_1b_up_proj.md")
+STAGE_KERNELS = {"hessian": ["hessian_pair_kernel", "hessian_reduce_kernel"],
+                 "scale_search": ["scale_search_kernel"], "lsq_fwd_bwd": ["lsq_kernel"],
+                 "pack_w4a16": ["pack_w4a16_kernel"]}
+
+
+def source_hash() -> str:
+    """Hash of the CUDA sources, matching the one recorded with the ncu traffic table."""
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "int4_group_wise_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        h.update(f.encode())
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_traffic(config: int):
+    """Per-stage DRAM bytes per launch from the committed ncu table, or {} when stale or absent."""
+    if config != 1 or not os.path.exists(TRAFFIC_FILE):
+        return {}
+    text = open(TRAFFIC_FILE).read()
+    recorded = next((ln.split(":", 1)[1].strip() for ln in text.splitlines() if ln.startswith("source_hash:")), None)
+    if recorded != source_hash():
+        return {}
+    per_kernel = {}
+    for ln in text.splitlines():
+        f = [x.strip() for x in ln.strip().strip("|").split("|")]
+        if len(f) == 2 and f[1].isdigit():
+            per_kernel[f[0]] = int(f[1])
+    return {st: sum(per_kernel.get(k, 0) for k in ks) for st, ks in STAGE_KERNELS.items()
+            if all(k in per_kernel for k in ks)}
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -274,6 +309,7 @@ def run_ours(args):
 
     if rank == 0:
         clocks = clk.summary()
+        traffic = load_traffic(args.config)
         hbm = float(peaks["hbm_gbs"])
         tc_peak = float(peaks["bf16_tflops"])
         sm_max = float(peaks.get("sm_max_mhz", 1965.0))
@@ -301,6 +337,8 @@ def run_ours(args):
                                         "bytes_per_launch": PACK_BYTES_PER_ELT * R * C,
                                         "peak_kind": f"{peak_kind} copy"}},
         }
+        for st_name, line_st in stage_lines.items():
+            line_st["roofline"]["traffic"] = traffic.get(st_name)
         dominant = max(stages, key=lambda s: mean[s])
         dom = stage_lines[dominant]["roofline"]
         if dominant == "hessian":
@@ -323,7 +361,8 @@ def run_ours(args):
                        "l2": "flushed (512 MB read sweep) before every stage; flush time in ms_per_step only"},
             "roofline": {"kernel": dominant, "bound": dom["bound"], "achieved": achieved, "peak": dom_peak,
                          "unit": roof_unit, "frac": achieved / dom_peak,
-                         "traffic": None, "peak_kind": dom["peak_kind"]},
+                         "traffic": traffic.get(dominant), "traffic_unit": "bytes per launch (ncu DRAM read + write)",
+                         "peak_kind": dom["peak_kind"]},
             "stages": stage_lines,
             "e2e": {"value": job_e2e_bytes / job_e2e_ms / 1e6, "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
