@@ -109,67 +109,85 @@ lsq_kernel(const float* __restrict__ W, const float* __restrict__ delta,
     }
 }
 
-// Four codes of one group as the low nibbles of 1.5*2^23 + q.
+// Eight codes of one group as the low nibbles of 1.5*2^23 + q, packed into a
+// 32-bit word (element 0 in the lowest nibble).
 // q = clamp(rint(w / d), -8, 7) is formed from r = w * (1/d): with both
 // roundings r lies within 3 ulp of the IEEE quotient, so clamping r to
 // [-8, 7] and rounding it (x + 1.5*2^23, which rounds to an integer in the
 // last place) gives the same integer unless r lands within 2^-18 of a
 // half-integer; then -- or when 1/d is not finite -- the IEEE division is
-// redone for the four elements.  For -8 <= q <= 7 the bit pattern of
+// redone for the eight elements.  For -8 <= q <= 7 the bit pattern of
 // 1.5*2^23 + q is 0x4B400000 + q, whose low nibble is q in 4-bit two's
-// complement.
-__device__ __forceinline__ uint32_t pack4(float4 w, float d) {
+// complement.  The arithmetic runs on packed FP32x2 pairs.
+__device__ __forceinline__ uint32_t pack8(float4 a, float4 b, float d) {
     constexpr float kM = 12582912.0f;                       // 1.5 * 2^23
     constexpr float kWin = 0.5f - 3.814697265625e-06f;      // 0.5 - 2^-18
     const float rc = __frcp_rn(d);
     bool slow = !(fabsf(rc) <= 3.4028234663852886e38f);
-    float t[4];
-    const float wv[4] = {w.x, w.y, w.z, w.w};
+    const float2 rc2 = make_float2(rc, rc);
+    const float2 M2 = make_float2(kM, kM);
+    const float2 negM2 = make_float2(-kM, -kM);
+    const float2 neg1 = make_float2(-1.0f, -1.0f);
+    const float2 w[4] = {make_float2(a.x, a.y), make_float2(a.z, a.w), make_float2(b.x, b.y), make_float2(b.z, b.w)};
+    float2 t[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
-        const float r = fminf(fmaxf(__fmul_rn(wv[e], rc), kQmin), kQmax);
-        t[e] = __fadd_rn(r, kM);
-        slow |= !(fabsf(__fsub_rn(r, __fsub_rn(t[e], kM))) <= kWin);
+        float2 r = __fmul2_rn(w[e], rc2);
+        r.x = fminf(fmaxf(r.x, kQmin), kQmax);
+        r.y = fminf(fmaxf(r.y, kQmin), kQmax);
+        t[e] = __fadd2_rn(r, M2);
+        const float2 f = __ffma2_rn(__fadd2_rn(t[e], negM2), neg1, r);   // r - q
+        slow |= !(fabsf(f.x) <= kWin) || !(fabsf(f.y) <= kWin);
     }
     if (slow) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) t[e] = __fadd_rn(code_of(scaled_exact(wv[e], d)), kM);
+        for (int e = 0; e < 4; ++e) {
+            t[e].x = __fadd_rn(code_of(scaled_exact(w[e].x, d)), kM);
+            t[e].y = __fadd_rn(code_of(scaled_exact(w[e].y, d)), kM);
+        }
     }
-    return (__float_as_uint(t[0]) & 0xFu) | ((__float_as_uint(t[1]) & 0xFu) << 4) |
-           ((__float_as_uint(t[2]) & 0xFu) << 8) | ((__float_as_uint(t[3]) & 0xFu) << 12);
+    uint32_t out = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        out |= (__float_as_uint(t[e].x) & 0xFu) << (8 * e);
+        out |= (__float_as_uint(t[e].y) & 0xFu) << (8 * e + 4);
+    }
+    return out;
 }
 
-// W4A16 export.  Lane l converts the float4 at elements 4l..4l+3 of a
-// 128-element step into two bytes (one coalesced 2-byte store); lanes 0, 8,
-// 16, 24 also write their group's binary16 scale.
-template <int U = 4>
+// W4A16 export.  A warp step covers 256 consecutive weights; lane l converts
+// weights 8l..8l+7 (one group is four lanes, so one reciprocal per lane) into
+// one 32-bit word, and the warp stores 128 contiguous bytes.  Lanes 0, 4, ...,
+// 28 also write their group's binary16 scale.  U steps in flight per warp.
+template <int U = 2>
 __global__ void __launch_bounds__(kStreamThreads)
-pack_w4a16_kernel(const float* __restrict__ W, const float* __restrict__ delta, int64_t nquads,
-                  uint16_t* __restrict__ packed16, uint16_t* __restrict__ scales) {
+pack_w4a16_kernel(const float* __restrict__ W, const float* __restrict__ delta, int64_t noct,
+                  uint32_t* __restrict__ packed32, uint16_t* __restrict__ scales) {
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kStreamThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kStreamThreads) >> 5;
-    const int64_t nsteps_ceil = (nquads + 31) >> 5;
+    const int64_t nsteps_ceil = (noct + 31) >> 5;    // noct = number of 8-weight octets
     for (int64_t s0 = warp * U; s0 < nsteps_ceil; s0 += nwarps * U) {
-        float4 w[U];
+        float4 wa[U], wb[U];
         float d[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t quad = (s0 + u) * 32 + lane;
-            if (quad < nquads) {
-                w[u] = __ldcs(reinterpret_cast<const float4*>(W) + quad);
-                d[u] = __ldg(delta + (quad >> 3));
+            const int64_t oct = (s0 + u) * 32 + lane;
+            if (oct < noct) {
+                wa[u] = __ldcs(reinterpret_cast<const float4*>(W) + 2 * oct);
+                wb[u] = __ldcs(reinterpret_cast<const float4*>(W) + 2 * oct + 1);
+                d[u] = __ldg(delta + (oct >> 2));
             } else {
-                w[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                wa[u] = wb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
                 d[u] = 0.f;
             }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const int64_t quad = (s0 + u) * 32 + lane;
-            if (quad < nquads) {
-                packed16[quad] = static_cast<uint16_t>(pack4(w[u], d[u]));
-                if ((lane & 7) == 0) scales[quad >> 3] = __half_as_ushort(__float2half_rn(d[u]));
+            const int64_t oct = (s0 + u) * 32 + lane;
+            if (oct < noct) {
+                __stcs(packed32 + oct, pack8(wa[u], wb[u], d[u]));
+                if ((lane & 3) == 0) scales[oct >> 2] = __half_as_ushort(__float2half_rn(d[u]));
             }
         }
     }

@@ -182,7 +182,7 @@ qat4_status qat4_scale_search(const float* W, int64_t R, int64_t C, const float*
     {
         std::lock_guard<std::mutex> lock(g_mutex);
         if (!info->search_attr) {
-            if (cudaFuncSetAttribute(qat4::scale_search_kernel<3>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            if (cudaFuncSetAttribute(qat4::scale_search_kernel<3, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(sizeof(qat4::SearchSmem))) != cudaSuccess)
                 return QAT4_ERR_CUDA;
             info->search_attr = true;
@@ -190,7 +190,7 @@ qat4_status qat4_scale_search(const float* W, int64_t R, int64_t C, const float*
     }
     const dim3 grid(static_cast<unsigned>((R + qat4::kSearchThreads - 1) / qat4::kSearchThreads),
                     static_cast<unsigned>(C / 32));
-    qat4::scale_search_kernel<3><<<grid, qat4::kSearchThreads, sizeof(qat4::SearchSmem), stream>>>(
+    qat4::scale_search_kernel<3, 1><<<grid, qat4::kSearchThreads, sizeof(qat4::SearchSmem), stream>>>(
         W, static_cast<int>(R), static_cast<int>(C), H, ldh, alpha, K, delta, idx, best_err);
     return launch_status();
 }
@@ -261,9 +261,9 @@ qat4_status qat4_pack_w4a16(const float* W, const float* delta, int64_t R, int64
     int dev;
     DeviceInfo* info;
     if (!device_info(&dev, &info)) return QAT4_ERR_CUDA;
-    const int64_t nquads = R * C / 4;
-    qat4::pack_w4a16_kernel<4><<<stream_blocks(nquads, info->sms, 4), qat4::kStreamThreads, 0, stream>>>(
-        W, delta, nquads, reinterpret_cast<uint16_t*>(packed), scales);
+    const int64_t noct = R * C / 8;   // C % 32 == 0: octets never straddle a group
+    qat4::pack_w4a16_kernel<2><<<stream_blocks(noct, info->sms, 2), qat4::kStreamThreads, 0, stream>>>(
+        W, delta, noct, reinterpret_cast<uint32_t*>(packed), scales);
     return launch_status();
 }
 

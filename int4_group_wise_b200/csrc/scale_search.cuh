@@ -111,36 +111,48 @@ __device__ __forceinline__ void group_error(const float (&w)[32], float dk, floa
 }
 
 // Two candidates at once: element j of the pair register holds (e0_j, e1_j);
-// one packed FMA (FFMA2) advances both candidates' row sums.
-template <int P>
-__device__ __forceinline__ void tri_ffma2(float2 h, const float2 (&e)[32], float2& t, float2& E) {
+// one packed FMA (FFMA2) advances both candidates' row sums.  Each row sum is
+// split into NCH interleaved chains (j - i mod NCH) so consecutive FFMA2s do
+// not wait on each other; the chains are added at the end of the row.  (The
+// screening bound holds for any summation order of these <= 33-term sums.)
+template <int NCH, int P>
+__device__ __forceinline__ void tri_ffma2(float2 h, const float2 (&e)[32], float2 (&t)[NCH], float2& E) {
     constexpr int i = tri_row(P);
     constexpr int j = tri_col(P);
-    t = __ffma2_rn(h, e[j], t);
+    constexpr int c = (j - i) % NCH;
+    t[c] = __ffma2_rn(h, e[j], t[c]);
     if constexpr (j == 31) {
-        E = __ffma2_rn(e[i], t, E);
-        t = make_float2(0.0f, 0.0f);
+        float2 r = t[0];
+#pragma unroll
+        for (int x = 1; x < NCH; ++x) r = __fadd2_rn(r, t[x]);
+        E = __ffma2_rn(e[i], r, E);
+#pragma unroll
+        for (int x = 0; x < NCH; ++x) t[x] = make_float2(0.0f, 0.0f);
     }
 }
 
-template <int Q2>
-__device__ __forceinline__ void tri_pair2(const float4* h32, const float2 (&e)[32], float2& t, float2& E) {
+template <int NCH, int Q2>
+__device__ __forceinline__ void tri_pair2(const float4* h32, const float2 (&e)[32], float2 (&t)[NCH], float2& E) {
     const float4 h = h32[Q2];                     // (h_p, h_p, h_p+1, h_p+1)
-    tri_ffma2<2 * Q2 + 0>(make_float2(h.x, h.y), e, t, E);
-    tri_ffma2<2 * Q2 + 1>(make_float2(h.z, h.w), e, t, E);
+    tri_ffma2<NCH, 2 * Q2 + 0>(make_float2(h.x, h.y), e, t, E);
+    tri_ffma2<NCH, 2 * Q2 + 1>(make_float2(h.z, h.w), e, t, E);
 }
 
-template <int... Q2s>
+template <int NCH, int... Q2s>
 __device__ __forceinline__ float2 quad_form_pair_impl(std::integer_sequence<int, Q2s...>, const float4* h32,
                                                       const float2 (&e)[32]) {
-    float2 t = make_float2(0.0f, 0.0f), E = make_float2(0.0f, 0.0f);
-    (tri_pair2<Q2s>(h32, e, t, E), ...);
+    float2 t[NCH];
+#pragma unroll
+    for (int x = 0; x < NCH; ++x) t[x] = make_float2(0.0f, 0.0f);
+    float2 E = make_float2(0.0f, 0.0f);
+    (tri_pair2<NCH, Q2s>(h32, e, t, E), ...);
     return E;
 }
 
 // float32 screening values of two candidates, E.x and E.y.
+template <int NCH>
 __device__ __forceinline__ float2 quad_form_pair(const float4* h32, const float2 (&e)[32]) {
-    return quad_form_pair_impl(std::make_integer_sequence<int, kTri / 2>{}, h32, e);
+    return quad_form_pair_impl<NCH>(std::make_integer_sequence<int, kTri / 2>{}, h32, e);
 }
 
 // Error vectors of two candidates (dk.x, dk.y) in packed form; every
@@ -218,7 +230,7 @@ struct TopK4 {
     }
 };
 
-template <int MINB>
+template <int MINB, int NCH>
 __global__ void __launch_bounds__(kSearchThreads, MINB)
 scale_search_kernel(const float* __restrict__ W, int R, int C,
                     const float* __restrict__ H, int64_t ldh,
@@ -309,7 +321,7 @@ scale_search_kernel(const float* __restrict__ W, int R, int C,
         const float2 dk = make_float2(__fmul_rn(__ldg(alpha + k), base), __fmul_rn(__ldg(alpha + k1), base));
         float2 e[32];
         group_error_pair(w2, dk, e, wslot, eslot);
-        const float2 E = quad_form_pair(sm.h32, e);
+        const float2 E = quad_form_pair<NCH>(sm.h32, e);
         float S0 = 0.0f, S1 = 0.0f;
 #pragma unroll
         for (int v = 0; v < 8; ++v) {
