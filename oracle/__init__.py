@@ -34,9 +34,13 @@ def lib():
         L.oracle_lsq_bwd.argtypes = [_P, _P, _P, ct.c_int, _I64, _I64, ct.c_float, _P, _P]
         L.oracle_pack_w4a16.argtypes = [_P, _P, _I64, _I64, _P, _P]
         L.oracle_codes.argtypes = [_P, _P, _I64, _I64, _P]
+        L.oracle_lsq_fwd_rowwise.argtypes = [_P, _P, _I64, _I64, _P]
+        L.oracle_lsq_bwd_rowwise.argtypes = [_P, _P, _P, ct.c_int, _I64, _I64, ct.c_float, _P, _P]
+        L.oracle_pack_w4a16_rowwise.argtypes = [_P, _P, _I64, _I64, _P, _P]
         for f in ("oracle_hessian", "oracle_hessian_entries", "oracle_hessian_block",
                   "oracle_scale_search", "oracle_lsq_fwd", "oracle_lsq_bwd",
-                  "oracle_pack_w4a16", "oracle_codes"):
+                  "oracle_pack_w4a16", "oracle_codes", "oracle_lsq_fwd_rowwise",
+                  "oracle_lsq_bwd_rowwise", "oracle_pack_w4a16_rowwise"):
             getattr(L, f).restype = None
     return _LIB
 
@@ -139,3 +143,39 @@ def codes(W: np.ndarray, delta: np.ndarray) -> np.ndarray:
     out = np.empty((R, C), np.int8)
     lib().oracle_codes(_p(W), _p(delta), R, C, _p(out))
     return out
+
+
+# ---------------------------------------------------------------- per-channel
+def lsq_fwd_rowwise(W: np.ndarray, delta: np.ndarray) -> np.ndarray:
+    """Q with one scale per row: delta float32 [R]."""
+    W = _c(W, np.float32)
+    delta = _c(delta, np.float32).reshape(-1)
+    R, C = W.shape
+    Q = np.empty_like(W)
+    lib().oracle_lsq_fwd_rowwise(_p(W), _p(delta), R, C, _p(Q))
+    return Q
+
+
+def lsq_bwd_rowwise(W: np.ndarray, delta: np.ndarray, G: np.ndarray, grad_scale: float):
+    """Returns (grad_W f32 [R, C], grad_delta f64 [R])."""
+    W = _c(W, np.float32)
+    delta = _c(delta, np.float32).reshape(-1)
+    is_bf16 = np.asarray(G).dtype == np.uint16
+    G = _c(G, np.uint16 if is_bf16 else np.float32)
+    R, C = W.shape
+    gW = np.empty_like(W)
+    gD = np.empty(R, np.float64)
+    lib().oracle_lsq_bwd_rowwise(_p(W), _p(delta), _p(G), int(is_bf16), R, C, ct.c_float(grad_scale),
+                                 _p(gW), _p(gD))
+    return gW, gD
+
+
+def pack_w4a16_rowwise(W: np.ndarray, delta: np.ndarray):
+    """Returns (packed uint8 [R, C/2], scale16 bits uint16 [R])."""
+    W = _c(W, np.float32)
+    delta = _c(delta, np.float32).reshape(-1)
+    R, C = W.shape
+    packed = np.empty((R, C // 2), np.uint8)
+    s16 = np.empty(R, np.uint16)
+    lib().oracle_pack_w4a16_rowwise(_p(W), _p(delta), R, C, _p(packed), _p(s16))
+    return packed, s16

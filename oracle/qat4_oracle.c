@@ -307,3 +307,61 @@ void oracle_codes(const float *W, const float *delta, int64_t R, int64_t C, int8
         for (int64_t c = 0; c < C; ++c)
             codes[r * C + c] = (int8_t)code_of(scaled(W[r * C + c], delta[r * G + c / GROUP]));
 }
+
+/* ------------------------------------------------ per-channel (one scale per row)
+ * Model card "Opt.Gear-1B-qat-int4-per-channel-unquantized": the same
+ * symmetric INT4 grid with one scale per output channel (row), W4A16 export
+ * with learned channel-wise scales.  The quantizer, the straight-through
+ * weight gradient and the step gradient are those of the group-32 functions
+ * above with the group widened to the whole row; the step-gradient
+ * normalisation uses the row's element count, s = 1/sqrt(C * 7), passed in.
+ * delta, grad_delta, scale16: one value per row [R]. */
+void oracle_lsq_fwd_rowwise(const float *W, const float *delta, int64_t R, int64_t C, float *Q)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t c = 0; c < C; ++c)
+            Q[r * C + c] = fake_quant(W[r * C + c], delta[r]);
+}
+
+void oracle_lsq_bwd_rowwise(const float *W, const float *delta, const void *Gp, int g_is_bf16,
+                            int64_t R, int64_t C, float grad_scale,
+                            float *grad_W, double *grad_delta)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        float dl = delta[r];
+        double acc = 0.0;
+        for (int64_t c = 0; c < C; ++c) {
+            int64_t idx = r * C + c;
+            float gi = g_is_bf16 ? bf16_to_float(((const uint16_t *)Gp)[idx])
+                                 : ((const float *)Gp)[idx];
+            float v = scaled(W[idx], dl);
+            int inside = (v >= QMIN) && (v <= QMAX);
+            grad_W[idx] = inside ? gi : 0.0f;
+            float d;
+            if (v <= QMIN)      d = QMIN;
+            else if (v >= QMAX) d = QMAX;
+            else                d = rintf(v) - v;
+            acc += (double)gi * (double)d;
+        }
+        grad_delta[r] = (double)grad_scale * acc;
+    }
+}
+
+void oracle_pack_w4a16_rowwise(const float *W, const float *delta, int64_t R, int64_t C,
+                               uint8_t *packed, uint16_t *scale16)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t j = 0; j < C / 2; ++j) {
+            int lo = (int)code_of(scaled(W[r * C + 2 * j], delta[r]));
+            int hi = (int)code_of(scaled(W[r * C + 2 * j + 1], delta[r]));
+            packed[r * (C / 2) + j] = (uint8_t)((lo & 0xF) | ((hi & 0xF) << 4));
+        }
+        _Float16 h = (_Float16)delta[r];
+        uint16_t bits;
+        memcpy(&bits, &h, sizeof bits);
+        scale16[r] = bits;
+    }
+}

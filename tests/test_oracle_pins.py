@@ -383,3 +383,52 @@ def test_pack_unpack_roundtrip_and_fp16(oracle_mod):
     p2, s2 = twin.pack(W, D)
     np.testing.assert_array_equal(packed, p2)
     np.testing.assert_array_equal(s16, s2)
+
+
+# ------------------------------------------------------------ per-channel variant
+
+def test_rowwise_lsq_hand_row(oracle_mod):
+    """One 64-weight row with the hand cases: grad_Delta = (sum of dQ/dDelta) / sqrt(64 * 7)."""
+    cases = _golden_rows("lsq_grad_cases.txt")
+    C, total = (int(x) if i == 0 else float(x) for i, x in enumerate(_golden_rows("lsq_grad_rowwise.txt")[0]))
+    v = np.zeros((1, C), f32)
+    v[0, :len(cases)] = [float(r[0]) for r in cases]
+    G = np.ones_like(v)
+    s = float(f32(1.0 / np.sqrt(C * 7)))
+    gW, gD = oracle_mod.lsq_bwd_rowwise(v, np.ones(1, f32), G, s)
+    assert abs(gD[0] - s * total) <= 1e-12 * abs(s * total)
+    np.testing.assert_array_equal(gW[0, :len(cases)], [float(r[1]) for r in cases])
+
+
+def test_rowwise_equals_group32_with_broadcast_scale(oracle_mod):
+    """A per-row scale broadcast to every group of the row reproduces the group-32 functions."""
+    rng = np.random.default_rng(21)
+    R, C = 9, 32 * 11
+    W = (rng.standard_normal((R, C)) * 0.02).astype(f32)
+    Dr = (np.abs(W).max(axis=1) / f32(7) * rng.uniform(0.4, 1.1, R)).astype(f32)
+    Dr[3] = 0                                   # Delta = 0 convention
+    Dg = np.repeat(Dr[:, None], C // 32, axis=1)
+    Gb = inputs.f32_to_bf16_bits((rng.standard_normal((R, C)) * 1e-3).astype(f32))
+    np.testing.assert_array_equal(_bits(oracle_mod.lsq_fwd_rowwise(W, Dr)), _bits(oracle_mod.lsq_fwd(W, Dg)))
+    s_row, s_grp = float(f32(1 / np.sqrt(C * 7))), float(f32(1 / np.sqrt(32 * 7)))
+    gWr, gDr = oracle_mod.lsq_bwd_rowwise(W, Dr, Gb, s_row)
+    gWg, gDg = oracle_mod.lsq_bwd(W, Dg, Gb, s_grp)
+    np.testing.assert_array_equal(_bits(gWr), _bits(gWg))
+    np.testing.assert_allclose(gDr / s_row, (gDg / s_grp).sum(axis=1), rtol=1e-12, atol=1e-300)
+    pr, sr = oracle_mod.pack_w4a16_rowwise(W, Dr)
+    pg, sg = oracle_mod.pack_w4a16(W, Dg)
+    np.testing.assert_array_equal(pr, pg)
+    np.testing.assert_array_equal(sr, sg[:, 0])
+    with np.errstate(over="ignore"):
+        np.testing.assert_array_equal(sr, Dr.astype(np.float16).view(np.uint16))
+
+
+def test_rowwise_single_group_row_is_group32(oracle_mod):
+    rng = np.random.default_rng(22)
+    W = (rng.standard_normal((7, 32)) * 0.02).astype(f32)
+    D = (np.abs(W).max(axis=1) / f32(7)).astype(f32)
+    G = (rng.standard_normal((7, 32)) * 1e-3).astype(f32)
+    gWr, gDr = oracle_mod.lsq_bwd_rowwise(W, D, G, S_LSQ)
+    gWg, gDg = oracle_mod.lsq_bwd(W, D[:, None], G, S_LSQ)
+    np.testing.assert_array_equal(gDr, gDg[:, 0])
+    np.testing.assert_array_equal(_bits(gWr), _bits(gWg))
