@@ -457,6 +457,70 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_per_channel(args):
+    """The per-channel variant (one scale per row) on the same layer shape: fused LSQ step and
+    W4A16 export, each launch timed with CUDA events after an L2 flush; one JSON line."""
+    import torch
+
+    import int4_group_wise_b200 as q4
+    from int4_group_wise_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_kind = load_peaks()
+    wl = inputs.workload(args.config)
+    m = wl.matrices[0]
+    W_h, G_h = wl.weight(m), wl.grad(m)
+    R, C = W_h.shape
+    W = torch.from_numpy(W_h).to(dev)
+    G = torch.from_numpy(G_h.view(np.int16)).to(dev).view(torch.bfloat16)
+    delta = (W.abs().amax(dim=1) / 7).contiguous()
+    Q, gW = torch.empty_like(W), torch.empty_like(W)
+    gD = torch.empty_like(delta)
+    packed = torch.empty((R, C // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((R,), dtype=torch.float16, device=dev)
+    flush_buf = torch.ones(128 << 20, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    lsq = lambda: q4.lsq_fwd_bwd_rowwise(W, delta, G, None, Q, gW, gD)
+    pack = lambda: q4.pack_w4a16_rowwise(W, delta, packed, scales)
+
+    def timed(fn, n):
+        ts = []
+        for _ in range(n):
+            torch.sum(flush_buf, dim=0, out=sink)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in ts) / n
+
+    for _ in range(args.warmup):
+        lsq()
+        pack()
+    q4.sync_check()
+    lsq_ms = timed(lsq, args.steps)
+    pack_ms = timed(pack, args.steps)
+    q4.sync_check()
+    lsq_bytes = (4 + 2 + 4 + 4) * R * C + 8 * R
+    pack_bytes = 4.5 * R * C + 6 * R
+    hbm = float(peaks["hbm_gbs"])
+    v_lsq, v_pack = lsq_bytes / lsq_ms / 1e6, pack_bytes / pack_ms / 1e6
+    print(json.dumps({
+        "metric": "per-channel LSQ fwd+bwd GB/s; per-channel W4A16 pack GB/s", "value": v_lsq, "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "higher_is_better": True,
+        "variant": "per-channel (one scale per row)", "data": "synthetic", "dtype": "f32",
+        "config": {"workload": f"W fp32 {R}x{C}, G bf16, one scale per row", "config_index": args.config,
+                   "l2": "flushed (512 MB read sweep) before every launch"},
+        "stages": {"lsq_fwd_bwd_rowwise": {"value": v_lsq, "unit": "GB/s", "ms": lsq_ms,
+                                           "bytes_per_launch": lsq_bytes, "frac": v_lsq / hbm},
+                   "pack_w4a16_rowwise": {"value": v_pack, "unit": "GB/s", "ms": pack_ms,
+                                          "bytes_per_launch": pack_bytes, "frac": v_pack / hbm}},
+        "peak": {"hbm_gbs": hbm, "kind": f"{peak_kind} copy"}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -465,11 +529,15 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--variant", choices=["group32", "per-channel"], default="group32",
+                    help="per-channel: time the one-scale-per-row LSQ step and export instead")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.variant == "per-channel":
+        run_per_channel(args)
     else:
         run_ours(args)
 

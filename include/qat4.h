@@ -188,6 +188,27 @@ qat4_status qat4_pack_w4a16(const float *W, const float *delta, int64_t R, int64
  *  Errors: QAT4_ERR_NULL, _SHAPE, _ALIGN, _WORKSPACE, _CUDA. */
 qat4_status qat4_hessian_noalloc(const uint16_t *X, int64_t n, int64_t C, float *H, cudaStream_t stream);
 
+/* ---------------------------------------------------------------- per-channel
+ * The same quantizer with one scale per output row (model card
+ * "Opt.Gear-1B-qat-int4-per-channel-unquantized": per-channel symmetric INT4
+ * weights with learned channel-wise scales, W4A16 export).  Arguments as for
+ * the group-32 calls, except that delta, grad_delta and scales hold one value
+ * per row ([R]), the step gradient of a row sums all C weights, and the
+ * normalisation passed in is normally grad_scale = 1/sqrt(C * 7).  The codes,
+ * Q, grad_W and packed bytes equal those of the group-32 calls given the row's
+ * scale in every group of the row.
+ *  Errors: QAT4_ERR_NULL, _SHAPE, _ALIGN, _DTYPE (LSQ backward), _CUDA. */
+qat4_status qat4_lsq_fwd_rowwise(const float *W, const float *delta, int64_t R, int64_t C,
+                                 float *Q, cudaStream_t stream);
+qat4_status qat4_lsq_bwd_rowwise(const float *W, const float *delta, const void *G, qat4_dtype g_dtype,
+                                 int64_t R, int64_t C, float grad_scale,
+                                 float *grad_W, float *grad_delta, cudaStream_t stream);
+qat4_status qat4_lsq_fwd_bwd_rowwise(const float *W, const float *delta, const void *G, qat4_dtype g_dtype,
+                                     int64_t R, int64_t C, float grad_scale,
+                                     float *Q, float *grad_W, float *grad_delta, cudaStream_t stream);
+qat4_status qat4_pack_w4a16_rowwise(const float *W, const float *delta, int64_t R, int64_t C,
+                                    uint8_t *packed, uint16_t *scales, cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the library's device error
  * word for the current device.  Returns QAT4_ERR_TIMEOUT if a kernel gave up
  * a bounded wait since the last check, QAT4_ERR_CUDA if synchronisation

@@ -40,6 +40,10 @@ EXPORTS = {
     "qat4_lsq_bwd": (ct.c_int, [_P, _P, _P, ct.c_int, _I64, _I64, _F, _P, _P, _P]),
     "qat4_lsq_fwd_bwd": (ct.c_int, [_P, _P, _P, ct.c_int, _I64, _I64, _F, _P, _P, _P, _P]),
     "qat4_pack_w4a16": (ct.c_int, [_P, _P, _I64, _I64, _P, _P, _P]),
+    "qat4_lsq_fwd_rowwise": (ct.c_int, [_P, _P, _I64, _I64, _P, _P]),
+    "qat4_lsq_bwd_rowwise": (ct.c_int, [_P, _P, _P, ct.c_int, _I64, _I64, _F, _P, _P, _P]),
+    "qat4_lsq_fwd_bwd_rowwise": (ct.c_int, [_P, _P, _P, ct.c_int, _I64, _I64, _F, _P, _P, _P, _P]),
+    "qat4_pack_w4a16_rowwise": (ct.c_int, [_P, _P, _I64, _I64, _P, _P, _P]),
     "qat4_sync_check": (ct.c_int, [_P]),
     "qat4_selftest_bounded_wait": (ct.c_int, [_I64, _P]),
 }
@@ -226,6 +230,72 @@ def pack_w4a16(W, delta, packed=None, scales=None, stream=None):
     scales = _out(scales, "scales", (R, C // 32), torch.float16, W)
     _check(L.qat4_pack_w4a16(_dev(W, "W"), _dev(delta, "delta"), R, C, _dev(packed, "packed"),
                              _dev(scales, "scales"), _stream(stream)), "qat4_pack_w4a16")
+    return packed, scales
+
+
+# ------------------------------------------------------------------ per-channel
+def rowwise_grad_scale(C: int) -> float:
+    """float32(1/sqrt(C * 7)): the per-channel step-gradient normalisation."""
+    return struct.unpack("<f", struct.pack("<f", 1.0 / math.sqrt(C * 7.0)))[0]
+
+
+def lsq_fwd_rowwise(W, delta, Q=None, stream=None):
+    """Q with one scale per row: delta float32 [R]."""
+    import torch
+    L = lib()
+    _dev(W, "W", torch.float32)
+    R, C = W.shape
+    _dev(delta, "delta", torch.float32, (R,))
+    Q = _out(Q, "Q", (R, C), torch.float32, W)
+    _check(L.qat4_lsq_fwd_rowwise(_dev(W, "W"), _dev(delta, "delta"), R, C, _dev(Q, "Q"), _stream(stream)),
+           "qat4_lsq_fwd_rowwise")
+    return Q
+
+
+def lsq_bwd_rowwise(W, delta, G, grad_scale=None, grad_W=None, grad_delta=None, stream=None):
+    import torch
+    L = lib()
+    _dev(W, "W", torch.float32)
+    R, C = W.shape
+    _dev(delta, "delta", torch.float32, (R,))
+    _dev(G, "G", None, (R, C))
+    gs = rowwise_grad_scale(C) if grad_scale is None else grad_scale
+    grad_W = _out(grad_W, "grad_W", (R, C), torch.float32, W)
+    grad_delta = _out(grad_delta, "grad_delta", (R,), torch.float32, W)
+    _check(L.qat4_lsq_bwd_rowwise(_dev(W, "W"), _dev(delta, "delta"), _dev(G, "G"), _gdtype(G), R, C,
+                                  ct.c_float(gs), _dev(grad_W, "grad_W"), _dev(grad_delta, "grad_delta"),
+                                  _stream(stream)), "qat4_lsq_bwd_rowwise")
+    return grad_W, grad_delta
+
+
+def lsq_fwd_bwd_rowwise(W, delta, G, grad_scale=None, Q=None, grad_W=None, grad_delta=None, stream=None):
+    import torch
+    L = lib()
+    _dev(W, "W", torch.float32)
+    R, C = W.shape
+    _dev(delta, "delta", torch.float32, (R,))
+    _dev(G, "G", None, (R, C))
+    gs = rowwise_grad_scale(C) if grad_scale is None else grad_scale
+    Q = _out(Q, "Q", (R, C), torch.float32, W)
+    grad_W = _out(grad_W, "grad_W", (R, C), torch.float32, W)
+    grad_delta = _out(grad_delta, "grad_delta", (R,), torch.float32, W)
+    _check(L.qat4_lsq_fwd_bwd_rowwise(_dev(W, "W"), _dev(delta, "delta"), _dev(G, "G"), _gdtype(G), R, C,
+                                      ct.c_float(gs), _dev(Q, "Q"), _dev(grad_W, "grad_W"),
+                                      _dev(grad_delta, "grad_delta"), _stream(stream)), "qat4_lsq_fwd_bwd_rowwise")
+    return Q, grad_W, grad_delta
+
+
+def pack_w4a16_rowwise(W, delta, packed=None, scales=None, stream=None):
+    """Returns (packed uint8 [R, C/2], scales float16 [R])."""
+    import torch
+    L = lib()
+    _dev(W, "W", torch.float32)
+    R, C = W.shape
+    _dev(delta, "delta", torch.float32, (R,))
+    packed = _out(packed, "packed", (R, C // 2), torch.uint8, W)
+    scales = _out(scales, "scales", (R,), torch.float16, W)
+    _check(L.qat4_pack_w4a16_rowwise(_dev(W, "W"), _dev(delta, "delta"), R, C, _dev(packed, "packed"),
+                                     _dev(scales, "scales"), _stream(stream)), "qat4_pack_w4a16_rowwise")
     return packed, scales
 
 

@@ -17,6 +17,7 @@
 #include "hessian.cuh"
 #include "lsq_pack.cuh"
 #include "scale_search.cuh"
+#include "rowwise.cuh"
 
 namespace {
 
@@ -264,6 +265,70 @@ qat4_status qat4_pack_w4a16(const float* W, const float* delta, int64_t R, int64
     const int64_t noct = R * C / 8;   // C % 32 == 0: octets never straddle a group
     qat4::pack_w4a16_kernel<2><<<stream_blocks(noct, info->sms, 2), qat4::kStreamThreads, 0, stream>>>(
         W, delta, noct, reinterpret_cast<uint32_t*>(packed), scales);
+    return launch_status();
+}
+
+// -------------------------------------------------------------- per-channel
+static qat4_status lsq_rowwise_common(const float* W, const float* delta, const void* G, qat4_dtype g_dtype,
+                                      int64_t R, int64_t C, float grad_scale, float* Q, float* grad_W,
+                                      float* grad_delta, bool fwd, bool bwd, cudaStream_t stream) {
+    if (!W || !delta || (fwd && !Q) || (bwd && (!G || !grad_W || !grad_delta))) return QAT4_ERR_NULL;
+    if (!valid_rc(R, C)) return QAT4_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(delta) || (fwd && !aligned16(Q)) ||
+        (bwd && (!aligned16(G) || !aligned16(grad_W) || !aligned16(grad_delta))))
+        return QAT4_ERR_ALIGN;
+    if (bwd && g_dtype != QAT4_F32 && g_dtype != QAT4_BF16) return QAT4_ERR_DTYPE;
+    const unsigned grid = static_cast<unsigned>(R);
+    const unsigned th = qat4::kRowThreads;
+    const int c = static_cast<int>(C);
+    if (fwd && !bwd) {
+        qat4::lsq_rowwise_kernel<float, true, false><<<grid, th, 0, stream>>>(W, delta, nullptr, c, 0.f, Q,
+                                                                             nullptr, nullptr);
+    } else if (g_dtype == QAT4_F32) {
+        const float* g = static_cast<const float*>(G);
+        if (fwd)
+            qat4::lsq_rowwise_kernel<float, true, true><<<grid, th, 0, stream>>>(W, delta, g, c, grad_scale, Q,
+                                                                                grad_W, grad_delta);
+        else
+            qat4::lsq_rowwise_kernel<float, false, true><<<grid, th, 0, stream>>>(W, delta, g, c, grad_scale,
+                                                                                 nullptr, grad_W, grad_delta);
+    } else {
+        const uint16_t* g = static_cast<const uint16_t*>(G);
+        if (fwd)
+            qat4::lsq_rowwise_kernel<uint16_t, true, true><<<grid, th, 0, stream>>>(W, delta, g, c, grad_scale,
+                                                                                   Q, grad_W, grad_delta);
+        else
+            qat4::lsq_rowwise_kernel<uint16_t, false, true><<<grid, th, 0, stream>>>(W, delta, g, c, grad_scale,
+                                                                                    nullptr, grad_W, grad_delta);
+    }
+    return launch_status();
+}
+
+qat4_status qat4_lsq_fwd_rowwise(const float* W, const float* delta, int64_t R, int64_t C, float* Q,
+                                 cudaStream_t stream) {
+    return lsq_rowwise_common(W, delta, nullptr, QAT4_F32, R, C, 0.f, Q, nullptr, nullptr, true, false, stream);
+}
+
+qat4_status qat4_lsq_bwd_rowwise(const float* W, const float* delta, const void* G, qat4_dtype g_dtype,
+                                 int64_t R, int64_t C, float grad_scale, float* grad_W, float* grad_delta,
+                                 cudaStream_t stream) {
+    return lsq_rowwise_common(W, delta, G, g_dtype, R, C, grad_scale, nullptr, grad_W, grad_delta, false, true,
+                              stream);
+}
+
+qat4_status qat4_lsq_fwd_bwd_rowwise(const float* W, const float* delta, const void* G, qat4_dtype g_dtype,
+                                     int64_t R, int64_t C, float grad_scale, float* Q, float* grad_W,
+                                     float* grad_delta, cudaStream_t stream) {
+    return lsq_rowwise_common(W, delta, G, g_dtype, R, C, grad_scale, Q, grad_W, grad_delta, true, true, stream);
+}
+
+qat4_status qat4_pack_w4a16_rowwise(const float* W, const float* delta, int64_t R, int64_t C, uint8_t* packed,
+                                    uint16_t* scales, cudaStream_t stream) {
+    if (!W || !delta || !packed || !scales) return QAT4_ERR_NULL;
+    if (!valid_rc(R, C)) return QAT4_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(delta) || !aligned16(packed) || !aligned16(scales)) return QAT4_ERR_ALIGN;
+    qat4::pack_w4a16_rowwise_kernel<<<static_cast<unsigned>(R), qat4::kRowThreads, 0, stream>>>(
+        W, delta, static_cast<int>(C), reinterpret_cast<uint32_t*>(packed), scales);
     return launch_status();
 }
 
