@@ -7,6 +7,9 @@
 // E(Delta) = e H_gg e^T with e = w_g - Q_Delta(w_g) and H_gg the 32x32 diagonal
 // block of H, over the candidates Delta_k = fl(alpha_k * fl(max|w_g| / 7)).
 //
+// The error vector is the exact difference e = w - Q_Delta(w) of the binary32
+// weights and their binary32 quantized values.
+//
 // Mapping: one CTA = one column group g x 128 rows; thread t owns row
 // r0 + t and keeps its 32 weights in registers.  H_gg is staged once per CTA
 // in shared memory as the upper triangle of H'_{ij} = H_ij + H_ji (j > i),
@@ -23,7 +26,8 @@
 // E is screened in float32 together with a rigorous bound
 //     |E32 - E| <= 80 u kappa S^2,   S = sum_i |e_i| sqrt|H_ii|,  u = 2^-24,
 // kappa = max(1, max_{i != j} |H_ij| / sqrt|H_ii H_jj|)  (= 1 for a PSD H)
-// which covers the 33-term FMA chains and the rounding of H'.  Every candidate
+// which covers the <= 33-term FMA sums (about 66u), the rounding of H' and of
+// the float32 difference fl(w - Q) used by the screen (about 3u).  Every candidate
 // whose interval [E32 - b, E32 + b] can still contain the minimum is
 // re-scored in float64 (the top four lower bounds are kept; if four or more
 // are undecided, all K candidates are re-scored), and the float64 minimum
@@ -192,11 +196,16 @@ __device__ __forceinline__ void group_error_pair(const float2 (&w2)[32], float2 
     }
 }
 
-// float64 value of one candidate (the re-score).
-__device__ __forceinline__ double quad_form64(const double* h64, const float (&e)[32]) {
+// float64 value of one candidate (the re-score): codes with the IEEE
+// division, Q = fl(dk * q), and the exact difference e = w - Q (exact in
+// binary64), summed in binary64.
+__device__ __forceinline__ double quad_form64(const double* h64, const float (&w)[32], float dk) {
     double ed[32];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) ed[i] = static_cast<double>(e[i]);
+    for (int i = 0; i < 32; ++i) {
+        const float q = code_of(scaled_exact(w[i], dk));
+        ed[i] = static_cast<double>(w[i]) - static_cast<double>(__fmul_rn(dk, q));
+    }
     double E = 0.0;
     int p = 0;
 #pragma unroll
@@ -355,9 +364,7 @@ scale_search_kernel(const float* __restrict__ W, int R, int C,
     const int count = overflow ? K : nfin;
     for (int a = 0; a < count; ++a) {
         const int kk = overflow ? a : (a == 0 ? top.k[0] : a == 1 ? top.k[1] : a == 2 ? top.k[2] : top.k[3]);
-        float e[32];
-        group_error(w, __fmul_rn(__ldg(alpha + kk), base), e, wslot, eslot);
-        const double E = quad_form64(sm.h64, e);
+        const double E = quad_form64(sm.h64, w, __fmul_rn(__ldg(alpha + kk), base));
         if (best_k < 0 || E < best || (E == best && kk < best_k)) { best = E; best_k = kk; }
     }
     delta_out[out] = __fmul_rn(__ldg(alpha + best_k), base);

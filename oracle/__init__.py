@@ -37,10 +37,11 @@ def lib():
         L.oracle_lsq_fwd_rowwise.argtypes = [_P, _P, _I64, _I64, _P]
         L.oracle_lsq_bwd_rowwise.argtypes = [_P, _P, _P, ct.c_int, _I64, _I64, ct.c_float, _P, _P]
         L.oracle_pack_w4a16_rowwise.argtypes = [_P, _P, _I64, _I64, _P, _P]
+        L.oracle_scale_search_rowwise.argtypes = [_P, _I64, _I64, _P, _I64, _P, ct.c_int32, _P, _P, _P, _P]
         for f in ("oracle_hessian", "oracle_hessian_entries", "oracle_hessian_block",
                   "oracle_scale_search", "oracle_lsq_fwd", "oracle_lsq_bwd",
                   "oracle_pack_w4a16", "oracle_codes", "oracle_lsq_fwd_rowwise",
-                  "oracle_lsq_bwd_rowwise", "oracle_pack_w4a16_rowwise"):
+                  "oracle_lsq_bwd_rowwise", "oracle_pack_w4a16_rowwise", "oracle_scale_search_rowwise"):
             getattr(L, f).restype = None
     return _LIB
 
@@ -179,3 +180,19 @@ def pack_w4a16_rowwise(W: np.ndarray, delta: np.ndarray):
     s16 = np.empty(R, np.uint16)
     lib().oracle_pack_w4a16_rowwise(_p(W), _p(delta), R, C, _p(packed), _p(s16))
     return packed, s16
+
+
+def scale_search_rowwise(W: np.ndarray, H: np.ndarray, alpha: np.ndarray, *, all_err: bool = False):
+    """Per-channel search with the full H.  Returns (delta f32 [R], idx i32 [R], best f64 [R][, all [R, K]])."""
+    W = _c(W, np.float32)
+    H = _c(H, np.float32)
+    alpha = _c(alpha, np.float32)
+    R, C = W.shape
+    K = alpha.size
+    delta = np.empty(R, np.float32)
+    idx = np.empty(R, np.int32)
+    best = np.empty(R, np.float64)
+    allv = np.empty((R, K), np.float64) if all_err else None
+    lib().oracle_scale_search_rowwise(_p(W), R, C, _p(H), H.shape[1], _p(alpha), K, _p(delta), _p(idx),
+                                      _p(best), _p(allv) if all_err else None)
+    return (delta, idx, best, allv) if all_err else (delta, idx, best)

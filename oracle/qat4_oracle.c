@@ -31,8 +31,9 @@
  *  fixed by the surviving text the plainest reading is taken:
  *    Q_Delta(w) = Delta * clamp(rint(w / Delta), -8, 7), rint = half-to-even;
  *    H = X^T X / n;  Delta_k = alpha_k * (max|w_g| / 7);
- *    objective per group = e H_gg e^T with e = w_g - Q(w_g) (block-diagonal
- *    reading of the objective, other groups held at zero error);
+ *    objective per group = e H_gg e^T with e = w_g - Q(w_g) exactly
+ *    (block-diagonal reading of the objective, other groups held at zero
+ *    error);
  *    LSQ (Esser et al., "Learned Step Size Quantization", ICLR 2020) step
  *    gradient with scale s = 1/sqrt(32 * 7).
  *
@@ -162,9 +163,10 @@ void oracle_hessian_block(const uint16_t *X, int64_t n, int64_t C,
  * is initialised as Delta* = argmin_Delta ||W X - Q_Delta(W) X||_F^2, searched
  * here over the finite grid Delta_k = alpha_k * (max|w_g| / 7).  For one
  * group g of row r the objective is the quadratic form e H_gg e^T with
- * e = w_g - Q_{Delta_k}(w_g) (computed as binary32 values, as the quantized
- * weights are stored) and H_gg the 32x32 diagonal block of H.  Every
- * candidate is evaluated; the smallest index reaching the minimum wins.
+ * e = w_g - Q_{Delta_k}(w_g), the exact difference of the binary32 weights and
+ * their binary32 quantized values (exact in binary64), and H_gg the 32x32
+ * diagonal block of H.  Every candidate is evaluated; the smallest index
+ * reaching the minimum wins.
  *
  * W: float [R, C] row-major; H: float, row stride ldh (only the diagonal
  * 32x32 blocks are read); alpha: float [K].
@@ -196,8 +198,7 @@ void oracle_scale_search(const float *W, int64_t R, int64_t C,
                 double e[GROUP];
                 for (int i = 0; i < GROUP; ++i) {
                     float qw = fake_quant(w[i], dk);
-                    float ei = w[i] - qw;
-                    e[i] = (double)ei;
+                    e[i] = (double)w[i] - (double)qw;   /* exact in binary64 */
                 }
                 double E = 0.0;
                 for (int i = 0; i < GROUP; ++i)
@@ -363,5 +364,51 @@ void oracle_pack_w4a16_rowwise(const float *W, const float *delta, int64_t R, in
         uint16_t bits;
         memcpy(&bits, &h, sizeof bits);
         scale16[r] = bits;
+    }
+}
+
+/* Per-channel scale search: the model card's objective
+ * Delta* = argmin ||W X - Q_Delta(W) X||_F^2 with one scale per row r, over the
+ * grid Delta_k = alpha_k * (max_c |w_rc| / 7).  The row's objective is the
+ * full quadratic form e H e^T, e = w_r - Q_{Delta_k}(w_r) (exact difference),
+ * summed in binary64 over all C x C entries of H (row stride ldh).
+ * Outputs per row [R]: delta, idx (smallest k on ties), best_err; all_err
+ * (nullable) [R, K]. */
+void oracle_scale_search_rowwise(const float *W, int64_t R, int64_t C,
+                                 const float *H, int64_t ldh,
+                                 const float *alpha, int32_t K,
+                                 float *delta_out, int32_t *idx_out, double *best_err,
+                                 double *all_err)
+{
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < R; ++r) {
+        const float *w = W + r * C;
+        float m = 0.0f;
+        for (int64_t i = 0; i < C; ++i) {
+            float a = fabsf(w[i]);
+            if (a > m) m = a;
+        }
+        float base = m / 7.0f;
+        double *e = (double *)__builtin_alloca((size_t)C * sizeof(double));
+        int32_t best_k = -1;
+        double best = 0.0;
+        float best_delta = 0.0f;
+        for (int32_t k = 0; k < K; ++k) {
+            float dk = alpha[k] * base;
+            for (int64_t i = 0; i < C; ++i) e[i] = (double)w[i] - (double)fake_quant(w[i], dk);
+            double E = 0.0;
+            for (int64_t i = 0; i < C; ++i)
+                for (int64_t j = 0; j < C; ++j)
+                    E += e[i] * (double)H[i * ldh + j] * e[j];
+            if (all_err) all_err[r * K + k] = E;
+            if (best_k < 0 || E < best) {
+                best = E;
+                best_k = k;
+                best_delta = dk;
+            }
+        }
+        delta_out[r] = best_delta;
+        idx_out[r] = best_k;
+        best_err[r] = best;
     }
 }

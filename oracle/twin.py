@@ -46,7 +46,7 @@ def search(W, H, alpha):
     base = (m / f32(7)).astype(f32)
     dk = (alpha[None, None, :] * base[:, :, None]).astype(f32)   # [R, G, K]
     q = fake_quant(Wg[:, :, None, :], dk[:, :, :, None])         # [R, G, K, 32]
-    e = (Wg[:, :, None, :] - q).astype(f32).astype(np.float64)
+    e = Wg[:, :, None, :].astype(np.float64) - q.astype(np.float64)     # exact difference
     Hb = np.stack([np.asarray(H, np.float64)[32 * g:32 * g + 32, 32 * g:32 * g + 32]
                    for g in range(G)])                           # [G, 32, 32]
     E = np.einsum("rgki,gij,rgkj->rgk", e, Hb, e)

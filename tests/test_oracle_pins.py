@@ -244,7 +244,7 @@ def test_search_objective_equals_output_error_from_X(oracle_mod):
             m = np.abs(w).max()
             for k in range(alpha.size):
                 dk = f32(alpha[k] * f32(m / f32(7)))
-                e = (w - twin.fake_quant(w, dk)).astype(np.float64)
+                e = w.astype(np.float64) - twin.fake_quant(w, dk).astype(np.float64)
                 direct = np.sum((Xd[:, 32 * g:32 * g + 32] @ e) ** 2) / n
                 assert abs(allE[r, g, k] - direct) <= 1e-12 * direct
             assert idx[r, g] == int(np.argmin(allE[r, g]))
@@ -265,7 +265,7 @@ def test_search_identity_hessian_is_mse(oracle_mod):
             mse = []
             for a in alpha:
                 d = f32(a * base)
-                e = (w - twin.fake_quant(w, d)).astype(np.float64)
+                e = w.astype(np.float64) - twin.fake_quant(w, d).astype(np.float64)
                 mse.append(float(e @ e))
             k = int(np.argmin(mse))
             assert idx[r, g] == k
@@ -332,6 +332,24 @@ def test_search_rtn_never_better_and_scale_covariance(oracle_mod):
     d4, i4, _ = oracle_mod.scale_search(W4, H, alpha)
     keep = [0, 2, 3]
     np.testing.assert_array_equal(d4[:, keep], delta[:, keep])
+
+
+def test_search_error_is_exact_difference(oracle_mod):
+    """Heavily clipped weights (|w| > 2|Q|) make the binary32 difference w - Q inexact; the
+    objective uses the exact difference (model-card objective on W - Q_Delta(W))."""
+    w = np.zeros((1, 32), f32)
+    w[0, 0] = f32(1.0)                         # sets the scale: base = fl(1/7)
+    w[0, 1] = f32(0.3333333432674408)          # moderate weight
+    w[0, 2] = f32(-1.0)
+    alpha = np.array([0.1], f32)               # Delta = 0.1/7: both +-1 clip at codes 7 / -8
+    H = np.eye(32, dtype=f32)
+    d, i, best, allE = oracle_mod.scale_search(w, H, alpha, all_err=True)
+    dk = f32(alpha[0] * f32(w[0, 0] / f32(7)))
+    Q = twin.fake_quant(w[0], dk)
+    e_exact = w[0].astype(np.float64) - Q.astype(np.float64)
+    assert allE[0, 0, 0] == float(e_exact @ e_exact)
+    e_f32 = (w[0] - Q).astype(np.float64)      # binary32 difference, rounded where clipped
+    assert float(e_f32 @ e_f32) != float(e_exact @ e_exact)
 
 
 def test_search_zero_group_and_twin(oracle_mod):
@@ -432,3 +450,47 @@ def test_rowwise_single_group_row_is_group32(oracle_mod):
     gWg, gDg = oracle_mod.lsq_bwd(W, D[:, None], G, S_LSQ)
     np.testing.assert_array_equal(gDr, gDg[:, 0])
     np.testing.assert_array_equal(_bits(gWr), _bits(gWg))
+
+
+def test_rowwise_search_pins(oracle_mod):
+    rng = np.random.default_rng(23)
+    alpha = inputs.alpha_grid(0.5, 0.01, 51)
+    # a one-group row is the group-32 search
+    W1 = (rng.standard_normal((6, 32)) * 0.02).astype(f32)
+    X1, X1b = _integer_calibration(rng, 64, 32)
+    H1 = oracle_mod.hessian(X1b).astype(f32)
+    d_r, i_r, b_r = oracle_mod.scale_search_rowwise(W1, H1, alpha)
+    d_g, i_g, b_g = oracle_mod.scale_search(W1, H1, alpha)
+    np.testing.assert_array_equal(i_r, i_g[:, 0])
+    np.testing.assert_array_equal(d_r, d_g[:, 0])
+    np.testing.assert_allclose(b_r, b_g[:, 0], rtol=1e-12)
+    # objective from X directly over the whole row (cross-group terms included)
+    R, C, n = 4, 96, 64
+    X, Xb = _integer_calibration(rng, n, C)
+    X[:, 40] += X[:, 70]                      # couples two groups
+    Xb = _bf16(X)
+    H = oracle_mod.hessian(Xb).astype(f32)
+    W = (rng.standard_normal((R, C)) * 0.02).astype(f32)
+    d, i, b, allE = oracle_mod.scale_search_rowwise(W, H, alpha, all_err=True)
+    Xd = X.astype(np.float64)
+    for r in range(R):
+        base = f32(np.abs(W[r]).max() / f32(7))
+        for k in range(0, alpha.size, 5):
+            dk = f32(alpha[k] * base)
+            e = W[r].astype(np.float64) - twin.fake_quant(W[r], dk).astype(np.float64)
+            direct = np.sum((Xd @ e) ** 2) / n
+            assert abs(allE[r, k] - direct) <= 1e-12 * direct
+        assert i[r] == int(np.argmin(allE[r]))
+    # H = I: plain squared error over the row
+    d0, i0, b0 = oracle_mod.scale_search_rowwise(W, np.eye(C, dtype=f32), alpha)
+    for r in range(R):
+        base = f32(np.abs(W[r]).max() / f32(7))
+        mse = [float(np.sum((W[r].astype(np.float64) - twin.fake_quant(W[r], f32(a * base)).astype(np.float64)) ** 2))
+               for a in alpha]
+        assert i0[r] == int(np.argmin(mse))
+    # weights on the alpha = 1 grid (power-of-two step) pick alpha = 1 with zero error
+    q = rng.integers(-6, 7, size=(3, 64)).astype(f32)
+    q[:, 5] = 7
+    Wg = (f32(2.0 ** -8) * q).astype(f32)
+    dg, ig, bg = oracle_mod.scale_search_rowwise(Wg, np.eye(64, dtype=f32) + f32(0.25), alpha)
+    assert np.all(ig == alpha.size - 1) and np.all(bg == 0) and np.all(dg == f32(2.0 ** -8))
