@@ -506,6 +506,38 @@ def run_per_channel(args):
     q4.sync_check()
     lsq_bytes = (4 + 2 + 4 + 4) * R * C + 8 * R
     pack_bytes = 4.5 * R * C + 6 * R
+
+    # per-channel scale search on the layer's Hessian (full C x C quadratic form per row)
+    X = torch.from_numpy(wl.activations(m.x_name).view(np.int16)).to(dev).view(torch.bfloat16)
+    H = q4.hessian(X)
+    del X
+    alpha_h = wl.alpha()
+    alpha = torch.from_numpy(alpha_h).to(dev)
+    sd = torch.empty((R,), dtype=torch.float32, device=dev)
+    si = torch.empty((R,), dtype=torch.int32, device=dev)
+    se = torch.empty((R,), dtype=torch.float32, device=dev)
+    ws = torch.empty(q4.lib().qat4_scale_search_rowwise_workspace_bytes(R, C), dtype=torch.uint8, device=dev)
+    search = lambda: q4.scale_search_rowwise(W, H, alpha, sd, si, se, ws)
+    search()
+    q4.sync_check()
+    search_ms = timed(search, 3)
+    q4.sync_check()
+    # code changes between consecutive candidates, from a 64-row sample (the sweep's work model)
+    rows = np.arange(0, R, max(1, R // 64))[:64]
+    Ws = W_h[rows]
+    bs = (np.abs(Ws).max(axis=1) / np.float32(7)).astype(np.float32)
+    prev, changes = None, 0
+    for a in alpha_h:
+        dk = (a * bs).astype(np.float32)[:, None]
+        qk = np.clip(np.rint(Ws / dk), -8, 7)
+        if prev is not None:
+            changes += int((qk != prev).sum())
+        prev = qk
+    changes_per_row = changes / len(rows)
+    K = alpha_h.size
+    dfma = 2.0 * R * C * C + R * changes_per_row * C + 3.0 * R * C * K
+    h_row_bytes = R * changes_per_row * C * 4.0
+    fp64_peak = 148 * 64 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
     hbm = float(peaks["hbm_gbs"])
     v_lsq, v_pack = lsq_bytes / lsq_ms / 1e6, pack_bytes / pack_ms / 1e6
     print(json.dumps({
@@ -517,7 +549,16 @@ def run_per_channel(args):
         "stages": {"lsq_fwd_bwd_rowwise": {"value": v_lsq, "unit": "GB/s", "ms": lsq_ms,
                                            "bytes_per_launch": lsq_bytes, "frac": v_lsq / hbm},
                    "pack_w4a16_rowwise": {"value": v_pack, "unit": "GB/s", "ms": pack_ms,
-                                          "bytes_per_launch": pack_bytes, "frac": v_pack / hbm}},
+                                          "bytes_per_launch": pack_bytes, "frac": v_pack / hbm},
+                   "scale_search_rowwise": {"value": R / search_ms * 1e3, "unit": "rows/s", "ms": search_ms,
+                                            "K": K, "code_changes_per_row": changes_per_row,
+                                            "fp64_fma_per_launch": dfma,
+                                            "fp64_frac": dfma / (search_ms * 1e-3) / fp64_peak,
+                                            "h_row_bytes_per_launch": h_row_bytes,
+                                            "h_row_gbs": h_row_bytes / search_ms / 1e6,
+                                            "note": "exact binary64 sweep; fp64_frac against 148 SM x 64 "
+                                                    "FP64 FMA/clock; the H rows re-read per code change "
+                                                    "come from L2"}},
         "peak": {"hbm_gbs": hbm, "kind": f"{peak_kind} copy"}}), flush=True)
 
 

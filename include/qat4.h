@@ -209,6 +209,28 @@ qat4_status qat4_lsq_fwd_bwd_rowwise(const float *W, const float *delta, const v
 qat4_status qat4_pack_w4a16_rowwise(const float *W, const float *delta, int64_t R, int64_t C,
                                     uint8_t *packed, uint16_t *scales, cudaStream_t stream);
 
+/* Per-channel scale search: for every row r and candidate
+ * Delta_k = fl(alpha[k] * fl(max_c |W[r,c]| / 7)) the full quadratic form
+ * E_k = e H e^T, e = w_r - Q_{Delta_k}(w_r) (exact difference), over all C x C
+ * entries of H (model card objective with one scale per row).
+ *  W          float32 [R, C], C <= 8192.
+ *  H          float32 [C, C], row stride ldh >= C; must be symmetric.
+ *  alpha, K   candidate multipliers, as for qat4_scale_search.
+ *  delta, idx, best_err   out [R]; idx is the argmin of E_k (smallest k on
+ *             ties); E_k is evaluated in binary64 (exact up to binary64
+ *             rounding and a dropped term below 1e-14 relative).
+ *  workspace  at least qat4_scale_search_rowwise_workspace_bytes(R, C) bytes
+ *             (16 R C + 4 R, rounded up): H w and H q for every row.  Large
+ *             matrices can be searched in row chunks to bound it.
+ *  Errors: QAT4_ERR_NULL, _SHAPE (C > 8192, ldh < C, K < 1), _ALIGN,
+ *  _WORKSPACE, _CUDA. */
+size_t qat4_scale_search_rowwise_workspace_bytes(int64_t R, int64_t C);
+qat4_status qat4_scale_search_rowwise(const float *W, int64_t R, int64_t C,
+                                      const float *H, int64_t ldh,
+                                      const float *alpha, int32_t K,
+                                      float *delta, int32_t *idx, float *best_err,
+                                      void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the library's device error
  * word for the current device.  Returns QAT4_ERR_TIMEOUT if a kernel gave up
  * a bounded wait since the last check, QAT4_ERR_CUDA if synchronisation

@@ -44,6 +44,8 @@ EXPORTS = {
     "qat4_lsq_bwd_rowwise": (ct.c_int, [_P, _P, _P, ct.c_int, _I64, _I64, _F, _P, _P, _P]),
     "qat4_lsq_fwd_bwd_rowwise": (ct.c_int, [_P, _P, _P, ct.c_int, _I64, _I64, _F, _P, _P, _P, _P]),
     "qat4_pack_w4a16_rowwise": (ct.c_int, [_P, _P, _I64, _I64, _P, _P, _P]),
+    "qat4_scale_search_rowwise_workspace_bytes": (_Z, [_I64, _I64]),
+    "qat4_scale_search_rowwise": (ct.c_int, [_P, _I64, _I64, _P, _I64, _P, _I32, _P, _P, _P, _P, _Z, _P]),
     "qat4_sync_check": (ct.c_int, [_P]),
     "qat4_selftest_bounded_wait": (ct.c_int, [_I64, _P]),
 }
@@ -297,6 +299,29 @@ def pack_w4a16_rowwise(W, delta, packed=None, scales=None, stream=None):
     _check(L.qat4_pack_w4a16_rowwise(_dev(W, "W"), _dev(delta, "delta"), R, C, _dev(packed, "packed"),
                                      _dev(scales, "scales"), _stream(stream)), "qat4_pack_w4a16_rowwise")
     return packed, scales
+
+
+def scale_search_rowwise(W, H, alpha, delta=None, idx=None, best_err=None, workspace=None, stream=None):
+    """Per-channel search with the full H.  Returns (delta f32 [R], idx i32 [R], best_err f32 [R])."""
+    import torch
+    L = lib()
+    _dev(W, "W", torch.float32)
+    R, C = W.shape
+    _dev(H, "H", torch.float32)
+    if H.dim() != 2 or H.shape[0] < C or H.shape[1] < C:
+        raise ValueError("H must be at least [C, C]")
+    _dev(alpha, "alpha", torch.float32)
+    delta = _out(delta, "delta", (R,), torch.float32, W)
+    idx = _out(idx, "idx", (R,), torch.int32, W)
+    best_err = _out(best_err, "best_err", (R,), torch.float32, W)
+    need = int(L.qat4_scale_search_rowwise_workspace_bytes(R, C))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=W.device)
+    _check(L.qat4_scale_search_rowwise(_dev(W, "W"), R, C, _dev(H, "H"), H.shape[1], _dev(alpha, "alpha"),
+                                       alpha.numel(), _dev(delta, "delta"), _dev(idx, "idx"),
+                                       _dev(best_err, "best_err"), _dev(workspace, "workspace", torch.uint8),
+                                       workspace.numel(), _stream(stream)), "qat4_scale_search_rowwise")
+    return delta, idx, best_err
 
 
 def sync_check(stream=None):

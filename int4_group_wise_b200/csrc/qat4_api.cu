@@ -18,6 +18,7 @@
 #include "lsq_pack.cuh"
 #include "scale_search.cuh"
 #include "rowwise.cuh"
+#include "rowwise_search.cuh"
 
 namespace {
 
@@ -34,6 +35,7 @@ struct DeviceInfo {
     int sms = 0;
     bool hessian_attr = false;
     bool search_attr = false;
+    bool rowsearch_attr = false;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mutex;
@@ -329,6 +331,59 @@ qat4_status qat4_pack_w4a16_rowwise(const float* W, const float* delta, int64_t 
     if (!aligned16(W) || !aligned16(delta) || !aligned16(packed) || !aligned16(scales)) return QAT4_ERR_ALIGN;
     qat4::pack_w4a16_rowwise_kernel<<<static_cast<unsigned>(R), qat4::kRowThreads, 0, stream>>>(
         W, delta, static_cast<int>(C), reinterpret_cast<uint32_t*>(packed), scales);
+    return launch_status();
+}
+
+size_t qat4_scale_search_rowwise_workspace_bytes(int64_t R, int64_t C) {
+    if (R < 1 || C < 32 || C % 32 != 0 || C > qat4::kRsMaxC) return 0;
+    const size_t hq = static_cast<size_t>(R) * static_cast<size_t>(C) * 2 * sizeof(double);
+    return hq + ((static_cast<size_t>(R) * sizeof(float) + 255) / 256) * 256;
+}
+
+qat4_status qat4_scale_search_rowwise(const float* W, int64_t R, int64_t C, const float* H, int64_t ldh,
+                                      const float* alpha, int32_t K, float* delta, int32_t* idx,
+                                      float* best_err, void* workspace, size_t workspace_bytes,
+                                      cudaStream_t stream) {
+    if (!W || !H || !alpha || !delta || !idx || !workspace) return QAT4_ERR_NULL;
+    if (!valid_rc(R, C) || C > qat4::kRsMaxC || K < 1 || ldh < C || R > (int64_t(1) << 22)) return QAT4_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(H) || !aligned16(alpha) || !aligned16(delta) || !aligned16(idx) ||
+        (best_err && !aligned16(best_err)) || !aligned16(workspace))
+        return QAT4_ERR_ALIGN;
+    if (workspace_bytes < qat4_scale_search_rowwise_workspace_bytes(R, C)) return QAT4_ERR_WORKSPACE;
+    const int ept = C <= 2048 ? 8 : (C <= 4096 ? 16 : 32);
+    const size_t smem = static_cast<size_t>(C) * (sizeof(double) + sizeof(uint32_t));
+    int dev;
+    DeviceInfo* info;
+    if (!device_info(&dev, &info)) return QAT4_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!info->rowsearch_attr) {
+            const int mx = static_cast<int>(qat4::kRsMaxC * (sizeof(double) + sizeof(uint32_t)));
+            if (cudaFuncSetAttribute(qat4::rowwise_sweep_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx) != cudaSuccess ||
+                cudaFuncSetAttribute(qat4::rowwise_sweep_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx) != cudaSuccess ||
+                cudaFuncSetAttribute(qat4::rowwise_sweep_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, mx) != cudaSuccess)
+                return QAT4_ERR_CUDA;
+            info->rowsearch_attr = true;
+        }
+    }
+    double* hbuf = static_cast<double*>(workspace);
+    double* tbuf = hbuf + R * C;
+    float* base = reinterpret_cast<float*>(tbuf + R * C);
+    const int r = static_cast<int>(R), c = static_cast<int>(C);
+    qat4::rowwise_base_kernel<<<static_cast<unsigned>((R * 32 + 255) / 256), 256, 0, stream>>>(W, r, c, base);
+    const dim3 g1(static_cast<unsigned>((C + qat4::kHqTile - 1) / qat4::kHqTile),
+                  static_cast<unsigned>((R + qat4::kHqTile - 1) / qat4::kHqTile));
+    qat4::rowwise_hq_kernel<<<g1, 256, 0, stream>>>(W, r, c, H, ldh, base, alpha, hbuf, tbuf);
+    const unsigned g2 = static_cast<unsigned>(R);
+    if (ept == 8)
+        qat4::rowwise_sweep_kernel<8><<<g2, qat4::kRsThreads, smem, stream>>>(W, c, H, ldh, alpha, K, base, hbuf, tbuf,
+                                                                            delta, idx, best_err);
+    else if (ept == 16)
+        qat4::rowwise_sweep_kernel<16><<<g2, qat4::kRsThreads, smem, stream>>>(W, c, H, ldh, alpha, K, base, hbuf, tbuf,
+                                                                             delta, idx, best_err);
+    else
+        qat4::rowwise_sweep_kernel<32><<<g2, qat4::kRsThreads, smem, stream>>>(W, c, H, ldh, alpha, K, base, hbuf, tbuf,
+                                                                             delta, idx, best_err);
     return launch_status();
 }
 
