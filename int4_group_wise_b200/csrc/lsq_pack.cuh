@@ -159,13 +159,13 @@ __device__ __forceinline__ uint32_t pack8(float4 a, float4 b, float d) {
 // weights 8l..8l+7 (one group is four lanes, so one reciprocal per lane) into
 // one 32-bit word, and the warp stores 128 contiguous bytes.  Lanes 0, 4, ...,
 // 28 also write their group's binary16 scale.  U steps in flight per warp.
-template <int U = 2>
-__global__ void __launch_bounds__(kStreamThreads)
+template <int U = 2, int NT = kStreamThreads>
+__global__ void __launch_bounds__(NT)
 pack_w4a16_kernel(const float* __restrict__ W, const float* __restrict__ delta, int64_t noct,
                   uint32_t* __restrict__ packed32, uint16_t* __restrict__ scales) {
     const int lane = threadIdx.x & 31;
-    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kStreamThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kStreamThreads) >> 5;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * NT + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * NT) >> 5;
     const int64_t nsteps_ceil = (noct + 31) >> 5;    // noct = number of 8-weight octets
     for (int64_t s0 = warp * U; s0 < nsteps_ceil; s0 += nwarps * U) {
         float4 wa[U], wb[U];

@@ -38,10 +38,12 @@ def lib():
         L.oracle_lsq_bwd_rowwise.argtypes = [_P, _P, _P, ct.c_int, _I64, _I64, ct.c_float, _P, _P]
         L.oracle_pack_w4a16_rowwise.argtypes = [_P, _P, _I64, _I64, _P, _P]
         L.oracle_scale_search_rowwise.argtypes = [_P, _I64, _I64, _P, _I64, _P, ct.c_int32, _P, _P, _P, _P]
+        L.oracle_w4a16_gemv.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P]
         for f in ("oracle_hessian", "oracle_hessian_entries", "oracle_hessian_block",
                   "oracle_scale_search", "oracle_lsq_fwd", "oracle_lsq_bwd",
                   "oracle_pack_w4a16", "oracle_codes", "oracle_lsq_fwd_rowwise",
-                  "oracle_lsq_bwd_rowwise", "oracle_pack_w4a16_rowwise", "oracle_scale_search_rowwise"):
+                  "oracle_lsq_bwd_rowwise", "oracle_pack_w4a16_rowwise", "oracle_scale_search_rowwise",
+                  "oracle_w4a16_gemv"):
             getattr(L, f).restype = None
     return _LIB
 
@@ -196,3 +198,15 @@ def scale_search_rowwise(W: np.ndarray, H: np.ndarray, alpha: np.ndarray, *, all
     lib().oracle_scale_search_rowwise(_p(W), R, C, _p(H), H.shape[1], _p(alpha), K, _p(delta), _p(idx),
                                       _p(best), _p(allv) if all_err else None)
     return (delta, idx, best, allv) if all_err else (delta, idx, best)
+
+
+def w4a16_gemv(x_bits: np.ndarray, packed: np.ndarray, scales16: np.ndarray, group: int) -> np.ndarray:
+    """y [M, R] (float64) = x @ (scale * code)^T from the packed export; x as bf16 bits [M, C]."""
+    x = _c(np.atleast_2d(x_bits), np.uint16)
+    packed = _c(packed, np.uint8)
+    scales16 = _c(scales16, np.uint16)
+    M, C = x.shape
+    R = packed.shape[0]
+    y = np.empty((M, R), np.float64)
+    lib().oracle_w4a16_gemv(_p(x), _p(packed), _p(scales16), M, R, C, int(group), _p(y))
+    return y

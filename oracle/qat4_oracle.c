@@ -412,3 +412,34 @@ void oracle_scale_search_rowwise(const float *W, int64_t R, int64_t C,
         best_err[r] = best;
     }
 }
+
+/* ------------------------------------------------------ W4A16 inference GEMV
+ * The consumer of the export ([card] "Quantization Configuration": W4A16,
+ * INT4 weights with 16-bit activations; "QAT Highlights": the same grid at
+ * export): y[m, r] = sum_c x[m, c] * (scale[r, c / group] * code[r, c]), with
+ * the binary16 scale and the 4-bit code of the packed layout (element 2j in the
+ * low nibble of byte j), x in bf16, products and sums in binary64.
+ * x: bf16 bits [M, C]; packed: uint8 [R, C/2]; scales: binary16 bits
+ * [R, C/group]; y: double [M, R]. */
+void oracle_w4a16_gemv(const uint16_t *x, const uint8_t *packed, const uint16_t *scales,
+                       int64_t M, int64_t R, int64_t C, int64_t group, double *y)
+{
+    const int64_t G = C / group;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r) {
+        for (int64_t m = 0; m < M; ++m) {
+            double s = 0.0;
+            for (int64_t c = 0; c < C; ++c) {
+                uint8_t byte = packed[r * (C / 2) + c / 2];
+                int nib = (c % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+                int code = nib >= 8 ? nib - 16 : nib;
+                _Float16 h;
+                uint16_t hb = scales[r * G + c / group];
+                memcpy(&h, &hb, sizeof h);
+                double w = (double)(float)h * (double)code;
+                s += (double)bf16_to_float(x[m * C + c]) * w;
+            }
+            y[m * R + r] = s;
+        }
+    }
+}

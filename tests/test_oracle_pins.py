@@ -494,3 +494,37 @@ def test_rowwise_search_pins(oracle_mod):
     Wg = (f32(2.0 ** -8) * q).astype(f32)
     dg, ig, bg = oracle_mod.scale_search_rowwise(Wg, np.eye(64, dtype=f32) + f32(0.25), alpha)
     assert np.all(ig == alpha.size - 1) and np.all(bg == 0) and np.all(dg == f32(2.0 ** -8))
+
+
+# ------------------------------------------------------------- W4A16 inference GEMV
+
+def test_w4a16_gemv_hand_row(oracle_mod):
+    rows = _golden_rows("w4a16_gemv.txt")
+    packed = np.array([[int(b, 16) for b in rows[0]]], np.uint8)
+    scale = np.array([[np.float16(float(rows[1][0])).view(np.uint16)]], np.uint16)
+    x = inputs.f32_to_bf16_bits(np.arange(1, 33, dtype=f32)[None, :])
+    y = oracle_mod.w4a16_gemv(x, packed, scale, 32)
+    assert y.shape == (1, 1) and y[0, 0] == float(rows[2][0])
+
+
+def test_w4a16_gemv_export_roundtrip_and_linearity(oracle_mod):
+    """Weights already on the exported grid (binary16-exact scale times a code) pack and
+    multiply back to x W^T exactly; the product is linear in x; both scale layouts agree."""
+    rng = np.random.default_rng(31)
+    R, C, M = 6, 128, 3
+    scale = rng.uniform(0.01, 0.05, (R, C // 32)).astype(np.float16).astype(f32)
+    codes = rng.integers(-8, 8, (R, C)).astype(f32)
+    W = (np.repeat(scale, 32, axis=1) * codes).astype(f32)          # exact
+    packed, s16 = oracle_mod.pack_w4a16(W, scale)
+    xf = inputs.bf16_bits_to_f32(inputs.f32_to_bf16_bits(rng.standard_normal((M, C)).astype(f32)))
+    xb = inputs.f32_to_bf16_bits(xf)
+    y = oracle_mod.w4a16_gemv(xb, packed, s16, 32)
+    np.testing.assert_allclose(y, xf.astype(np.float64) @ W.astype(np.float64).T, rtol=1e-13, atol=1e-13)
+    y2 = oracle_mod.w4a16_gemv(inputs.f32_to_bf16_bits(2 * xf), packed, s16, 32)
+    np.testing.assert_array_equal(y2, 2 * y)
+    # per-channel scales (group = C) through the row-wise export
+    rs = scale[:, 0]
+    Wr = (rs[:, None] * codes).astype(f32)
+    pr, sr = oracle_mod.pack_w4a16_rowwise(Wr, rs)
+    yr = oracle_mod.w4a16_gemv(xb, pr, sr, C)
+    np.testing.assert_allclose(yr, xf.astype(np.float64) @ Wr.astype(np.float64).T, rtol=1e-13, atol=1e-13)
