@@ -57,12 +57,16 @@ STAGE_KERNELS = {"hessian": ["hessian_pair_kernel", "hessian_reduce_kernel"],
                  "pack_w4a16": ["pack_w4a16_kernel"]}
 
 
+STEP_SOURCES = ("device_common.cuh", "hessian.cuh", "lsq_pack.cuh", "scale_search.cuh")
+
+
 def source_hash() -> str:
-    """Hash of the CUDA sources, matching the one recorded with the ncu traffic table."""
+    """Hash of the kernel sources of the group-32 step, matching the one recorded with the ncu
+    traffic table."""
     import hashlib
     h = hashlib.sha256()
     d = os.path.join(ROOT, "int4_group_wise_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in STEP_SOURCES:
         h.update(f.encode())
         with open(os.path.join(d, f), "rb") as fh:
             h.update(fh.read())
@@ -562,6 +566,107 @@ def run_per_channel(args):
         "peak": {"hbm_gbs": hbm, "kind": f"{peak_kind} copy"}}), flush=True)
 
 
+def run_w4a16_decode(args):
+    """Decode on the W4A16 export of the 8B-class stack (32 layers x {q, k, v, o, gate, up,
+    down}): one step = the 224 GEMVs of one token batch (M = 1 and M = 4), replayed from a CUDA
+    graph.  The seeded layer-0 weights, packed once, are copied into 32 distinct layer buffers
+    (3.9 GB of codes and scales, 31x L2), so every step streams its bytes from HBM."""
+    import torch
+
+    import int4_group_wise_b200 as q4
+    from int4_group_wise_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_kind = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    wl = inputs.workload(4)
+    layer0 = [m for m in wl.matrices if m.name.startswith("L0.")]
+    n_layers = len(wl.matrices) // len(layer0) if args.layers is None else args.layers
+    base = []
+    for m in layer0:
+        W = torch.from_numpy(wl.weight(m)).to(dev)
+        R, C = W.shape
+        delta = (W.abs().reshape(R, C // 32, 32).amax(dim=2) / 7).contiguous()
+        base.append(q4.pack_w4a16(W, delta))
+        del W, delta
+    q4.sync_check()
+    layers = [[(p.clone(), sc.clone()) for p, sc in base] for _ in range(n_layers)]
+    del base
+    torch.cuda.synchronize()
+    shapes = [(m.d_out, m.d_in) for m in layer0]
+    weights = sum(R * C for R, C in shapes) * n_layers
+    code_bytes = sum(R * C // 2 + R * (C // 32) * 2 for R, C in shapes) * n_layers
+    stream = torch.cuda.Stream(dev)
+    flush_buf = torch.ones(128 << 20, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    results = {}
+    for M in (1, 4):
+        xs = {C: torch.from_numpy(inputs.activations(M, C, seed=M, cfg=4, name=f"decode_x/{C}").view(np.int16))
+              .to(dev).view(torch.bfloat16) for C in sorted({C for _, C in shapes})}
+        ys = [torch.empty((M, R), dtype=torch.float32, device=dev) for R, _ in shapes]
+
+        def step():
+            for lay in layers:
+                for (R, C), (p, sc), y in zip(shapes, lay, ys):
+                    q4.w4a16_gemv(xs[C], p, sc, y, stream=stream)
+
+        with torch.cuda.stream(stream):
+            for _ in range(args.warmup):
+                step()
+        stream.synchronize()
+        q4.sync_check(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step()
+        for _ in range(args.warmup):
+            g.replay()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            b.record(stream)
+        torch.cuda.synchronize()
+        q4.sync_check(stream)
+        step_ms = a.elapsed_time(b) / args.steps
+        step_bytes = code_bytes + n_layers * sum(M * C * 2 + M * R * 4 for R, C in shapes)
+        # each shape on its own, L2 flushed before every launch (layer 0's buffers)
+        per_shape = {}
+        for m, (R, C), (p, sc), y in zip(layer0, shapes, layers[0], ys):
+            ts = []
+            with torch.cuda.stream(stream):
+                for _ in range(max(args.steps, 10)):
+                    torch.sum(flush_buf, dim=0, out=sink)
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    q4.w4a16_gemv(xs[C], p, sc, y, stream=stream)
+                    e1.record(stream)
+                    ts.append((e0, e1))
+            torch.cuda.synchronize()
+            us = 1e3 * sum(e0.elapsed_time(e1) for e0, e1 in ts) / len(ts)
+            nbytes = R * C // 2 + R * (C // 32) * 2 + M * C * 2 + M * R * 4
+            per_shape[m.name.split(".")[1]] = {"shape": [R, C], "us": us, "gbs": nbytes / us / 1e3,
+                                              "frac": nbytes / us / 1e3 / hbm}
+        del g
+        gbs = step_bytes / step_ms / 1e6
+        results[M] = {"tokens_per_s": M * 1e3 / step_ms, "ms_per_step": step_ms, "gbs": gbs, "frac": gbs / hbm,
+                      "bytes_per_step": step_bytes, "launches_per_step": len(shapes) * n_layers,
+                      "per_shape_l2_flushed": per_shape}
+    r1 = results[1]
+    print(json.dumps({
+        "metric": "W4A16 decode GEMV GB/s over the 8B-class stack (M = 1)", "value": r1["gbs"], "unit": "GB/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": r1["ms_per_step"],
+        "higher_is_better": True, "variant": "w4a16-decode", "data": "synthetic", "dtype": "bf16 x int4 -> f32",
+        "config": {"workload": f"8B-class stack, {n_layers} layers x 7 matrices, {weights} weights, "
+                               "group-32 export, decode batch M = 1 and 4",
+                   "l2": "inputs 31x L2 (distinct layer buffers); per-shape times flush L2 before every launch"},
+        "roofline": {"bound": "hbm", "achieved": r1["gbs"], "peak": hbm, "unit": "GB/s", "frac": r1["frac"],
+                     "peak_kind": f"{peak_kind} copy"},
+        "gpu_launches": r1["launches_per_step"] * args.steps,
+        "stages": {f"M={M}": v for M, v in results.items()}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -570,8 +675,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--variant", choices=["group32", "per-channel"], default="group32",
-                    help="per-channel: time the one-scale-per-row LSQ step and export instead")
+    ap.add_argument("--variant", choices=["group32", "per-channel", "w4a16-decode"], default="group32",
+                    help="per-channel: time the one-scale-per-row LSQ step and export instead; "
+                         "w4a16-decode: time the inference GEMV on the packed 8B-class stack")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="w4a16-decode: number of layers of the 8B-class stack (default: all 32)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -579,6 +687,8 @@ def main():
         run_reference(args)
     elif args.variant == "per-channel":
         run_per_channel(args)
+    elif args.variant == "w4a16-decode":
+        run_w4a16_decode(args)
     else:
         run_ours(args)
 

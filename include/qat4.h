@@ -231,6 +231,27 @@ qat4_status qat4_scale_search_rowwise(const float *W, int64_t R, int64_t C,
                                       float *delta, int32_t *idx, float *best_err,
                                       void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* ---------------------------------------------------------------- inference
+ * The product on the W4A16 export (model card "Opt.Gear-1B-qat-int4-per-
+ * channel-unquantized", section "Quantization Configuration": INT4 weights,
+ * 16-bit activations), for decode-sized batches:
+ *     y[m, r] = sum_c x[m, c] * (scale[r, c / group] * code[r, c])
+ *  x       bf16 bit patterns [M, C] (M tokens, 1 <= M <= 65535; processed up to four
+ *          tokens per pass -- fewer when x of a wide row does not fit shared memory -- so
+ *          the codes are read once per pass).
+ *  packed  uint8 [R, C/2], the layout of qat4_pack_w4a16 (element 2j in the low nibble of
+ *          byte j, 4-bit two's complement).
+ *  scales  binary16 bit patterns [R, C/group]: group = 32 for the export of
+ *          qat4_pack_w4a16, group = C for qat4_pack_w4a16_rowwise (any multiple of 32 that
+ *          divides C is accepted).
+ *  y       out float32 [M, R]; zeroed on the stream first, then written.  Products are
+ *          exact, sums float32 in an order fixed by (R, C, M) and the SM count.
+ *  C must be a multiple of 32 and small enough that one token's x (bf16) and two 32 KB
+ *  stages fit the opt-in shared memory of a block (C <= 83296 on B200); else _SHAPE.
+ *  Errors: QAT4_ERR_NULL, _SHAPE, _ALIGN, _CUDA. */
+qat4_status qat4_w4a16_gemv(const uint16_t *x, int64_t M, const uint8_t *packed, const uint16_t *scales,
+                            int64_t R, int64_t C, int64_t group, float *y, cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the library's device error
  * word for the current device.  Returns QAT4_ERR_TIMEOUT if a kernel gave up
  * a bounded wait since the last check, QAT4_ERR_CUDA if synchronisation

@@ -46,6 +46,7 @@ EXPORTS = {
     "qat4_pack_w4a16_rowwise": (ct.c_int, [_P, _P, _I64, _I64, _P, _P, _P]),
     "qat4_scale_search_rowwise_workspace_bytes": (_Z, [_I64, _I64]),
     "qat4_scale_search_rowwise": (ct.c_int, [_P, _I64, _I64, _P, _I64, _P, _I32, _P, _P, _P, _P, _Z, _P]),
+    "qat4_w4a16_gemv": (ct.c_int, [_P, _I64, _P, _P, _I64, _I64, _I64, _P, _P]),
     "qat4_sync_check": (ct.c_int, [_P]),
     "qat4_selftest_bounded_wait": (ct.c_int, [_I64, _P]),
 }
@@ -322,6 +323,29 @@ def scale_search_rowwise(W, H, alpha, delta=None, idx=None, best_err=None, works
                                        _dev(best_err, "best_err"), _dev(workspace, "workspace", torch.uint8),
                                        workspace.numel(), _stream(stream)), "qat4_scale_search_rowwise")
     return delta, idx, best_err
+
+
+def w4a16_gemv(x, packed, scales, y=None, stream=None):
+    """y [M, R] float32 = x @ (scale * code)^T on the packed export; x bf16 [M, C] (or [C]);
+    scales float16 [R, C/group] (group-32 export) or [R] (per-row export)."""
+    import torch
+    L = lib()
+    if x.dim() == 1:
+        x = x.unsqueeze(0)
+    _dev(x, "x", torch.bfloat16)
+    M, C = x.shape
+    _dev(packed, "packed", torch.uint8)
+    R = packed.shape[0]
+    if tuple(packed.shape) != (R, C // 2):
+        raise ValueError("packed must be [R, C/2]")
+    _dev(scales, "scales", torch.float16)
+    G = scales.numel() // R
+    if G < 1 or scales.numel() != R * G or C % G != 0:
+        raise ValueError("scales must hold C/group values per row")
+    y = _out(y, "y", (M, R), torch.float32, x)
+    _check(L.qat4_w4a16_gemv(_dev(x, "x"), M, _dev(packed, "packed"), _dev(scales, "scales"), R, C, C // G,
+                             _dev(y, "y"), _stream(stream)), "qat4_w4a16_gemv")
+    return y
 
 
 def sync_check(stream=None):

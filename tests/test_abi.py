@@ -83,3 +83,19 @@ def test_pack_search_hessian_validation():
     assert L.qat4_hessian(A, 64, 40, A, None, 0, None) == 2
     assert L.qat4_hessian(MIS, 64, 64, A, None, 0, None) == 3
     assert L.qat4_selftest_bounded_wait(0, None) == 2
+
+
+@pytest.mark.parametrize("args,code", [
+    ((None, 1, A, A, 8, 64, 32, A), 1),
+    ((A, 1, A, None, 8, 64, 32, A), 1),
+    ((A, 0, A, A, 8, 64, 32, A), 2),          # no token
+    ((A, 1, A, A, 8, 48, 32, A), 2),          # C not a multiple of 32
+    ((A, 1, A, A, 8, 64, 16, A), 2),          # group below 32
+    ((A, 1, A, A, 8, 96, 64, A), 2),          # group does not divide C
+    ((A, 1, A, A, 0, 64, 32, A), 2),
+    ((MIS, 1, A, A, 8, 64, 32, A), 3),
+    ((A, 1, A, MIS, 8, 64, 32, A), 3),
+])
+def test_w4a16_gemv_validation(args, code):
+    x, M, packed, scales, R, C, group, y = args
+    assert q4.lib().qat4_w4a16_gemv(x, M, packed, scales, R, C, group, y, None) == code
