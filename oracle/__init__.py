@@ -210,3 +210,28 @@ def w4a16_gemv(x_bits: np.ndarray, packed: np.ndarray, scales16: np.ndarray, gro
     y = np.empty((M, R), np.float64)
     lib().oracle_w4a16_gemv(_p(x), _p(packed), _p(scales16), M, R, C, int(group), _p(y))
     return y
+
+
+def fq_gemm(X_bits: np.ndarray, W: np.ndarray, delta: np.ndarray) -> np.ndarray:
+    """Y [T, R] (float64) = X @ bf16(Q_delta(W))^T; X as bf16 bits [T, C], W float32 [R, C],
+    delta float32 [R, C/32]."""
+    X = _c(np.atleast_2d(X_bits), np.uint16)
+    W = _c(W, np.float32)
+    delta = _c(delta, np.float32)
+    T, C = X.shape
+    R = W.shape[0]
+    Y = np.empty((T, R), np.float64)
+    lib().oracle_fq_gemm(_p(X), _p(W), _p(delta), T, R, C, _p(Y))
+    return Y
+
+
+def fq_gemm_entries(X_bits: np.ndarray, W: np.ndarray, delta: np.ndarray, tt, rr) -> np.ndarray:
+    """Y[tt[m], rr[m]] of fq_gemm (float64), for sampled checks of large outputs."""
+    X = _c(np.atleast_2d(X_bits), np.uint16)
+    W = _c(W, np.float32)
+    delta = _c(delta, np.float32)
+    tt = _c(tt, np.int64)
+    rr = _c(rr, np.int64)
+    out = np.empty(tt.size, np.float64)
+    lib().oracle_fq_gemm_entries(_p(X), _p(W), _p(delta), X.shape[1], tt.size, _p(tt), _p(rr), _p(out))
+    return out

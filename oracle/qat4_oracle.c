@@ -1,7 +1,8 @@
 /*
  * qat4_oracle.c -- plain CPU reference of the group-32 symmetric INT4 weight
  * quantizer (calibration Hessian, Hessian-weighted scale search, LSQ forward /
- * backward, W4A16 packing).
+ * backward, W4A16 packing), and the products either side of it (the W4A16
+ * inference GEMV on the export, the fake-quant forward GEMM of a QAT step).
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, loads or
  * calls this file; only the test suite, the smoke check and the benchmark's
@@ -44,6 +45,7 @@
  */
 #include <math.h>
 #include <stdint.h>
+#include <stdlib.h>
 #include <string.h>
 #ifdef _OPENMP
 #include <omp.h>
@@ -441,5 +443,63 @@ void oracle_w4a16_gemv(const uint16_t *x, const uint8_t *packed, const uint16_t 
             }
             y[m * R + r] = s;
         }
+    }
+}
+
+/* --------------------------------------------- fake-quant forward GEMM (QAT)
+ * The forward of a quantized linear layer in a QAT step ([blog] section 3
+ * "LSQ-based QAT": the forward pass runs on the weights projected onto the
+ * INT4 grid that deployment uses): Y = X * Qb^T with Q = Q_Delta(W) in binary32
+ * (as oracle_lsq_fwd) and Qb = Q rounded to bf16, round-to-nearest-even -- the
+ * operand precision of a bf16 matrix multiply, which the pages leave implicit
+ * (plainest reading: the usual bf16 mixed-precision forward).  Products and
+ * sums in binary64.
+ * X: bf16 bits [T, C]; W: float [R, C]; delta: float [R, C/32]; Y: double [T, R]. */
+
+/* float -> bf16 bits, round to nearest, ties to even (finite inputs only). */
+static uint16_t float_to_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7FFFu + lsb;
+    return (uint16_t)(u >> 16);
+}
+
+static double fq_operand(const float *W, const float *delta, int64_t C, int64_t r, int64_t c)
+{
+    float q = fake_quant(W[r * C + c], delta[r * (C / GROUP) + c / GROUP]);
+    return (double)bf16_to_float(float_to_bf16_rne(q));
+}
+
+void oracle_fq_gemm(const uint16_t *X, const float *W, const float *delta,
+                    int64_t T, int64_t R, int64_t C, double *Y)
+{
+    double *Qb = (double *)malloc((size_t)(R * C) * sizeof(double));
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t c = 0; c < C; ++c) Qb[r * C + c] = fq_operand(W, delta, C, r, c);
+    #pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t r = 0; r < R; ++r) {
+            double s = 0.0;
+            for (int64_t c = 0; c < C; ++c) s += (double)bf16_to_float(X[t * C + c]) * Qb[r * C + c];
+            Y[t * R + r] = s;
+        }
+    }
+    free(Qb);
+}
+
+/* Selected entries Y[tt[m], rr[m]] of the same product (for sampled checks of
+ * full-size outputs); out[m] in binary64. */
+void oracle_fq_gemm_entries(const uint16_t *X, const float *W, const float *delta, int64_t C,
+                            int64_t nsel, const int64_t *tt, const int64_t *rr, double *out)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < nsel; ++m) {
+        double s = 0.0;
+        for (int64_t c = 0; c < C; ++c)
+            s += (double)bf16_to_float(X[tt[m] * C + c]) * fq_operand(W, delta, C, rr[m], c);
+        out[m] = s;
     }
 }

@@ -9,7 +9,9 @@ small cases.  Same readings of the pages as the C oracle:
   Configuration", symmetric zero-point 0);
 * per-group objective e H_gg e^T over Delta_k = alpha_k * (max|w| / 7) (model
   card objective, block-diagonal reading);
-* LSQ gradients (blog section 3; Esser et al. 2020).
+* LSQ gradients (blog section 3; Esser et al. 2020);
+* the fake-quant forward product X @ bf16(Q)^T (blog section 3, bf16 operands,
+  round to nearest even).
 """
 from __future__ import annotations
 
@@ -77,3 +79,19 @@ def pack(W, delta):
     with np.errstate(over="ignore"):
         s16 = np.asarray(delta, f32).astype(np.float16).view(np.uint16)
     return packed, s16
+
+
+def _bf16_rne(a):
+    """float32 -> float32 holding the nearest bf16 value (ties to even), by integer rounding of
+    the bit pattern."""
+    u = np.asarray(a, f32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(f32)
+
+
+def fq_gemm(X, W, delta):
+    """X float32 (bf16-valued) [T, C], W [R, C], delta [R, C/32] -> float64 [T, R]."""
+    W = np.asarray(W, f32)
+    D = np.repeat(np.asarray(delta, f32), 32, axis=1)
+    Qb = _bf16_rne(fake_quant(W, D)).astype(np.float64)
+    return np.asarray(X, np.float64) @ Qb.T

@@ -528,3 +528,61 @@ def test_w4a16_gemv_export_roundtrip_and_linearity(oracle_mod):
     pr, sr = oracle_mod.pack_w4a16_rowwise(Wr, rs)
     yr = oracle_mod.w4a16_gemv(xb, pr, sr, C)
     np.testing.assert_allclose(yr, xf.astype(np.float64) @ Wr.astype(np.float64).T, rtol=1e-13, atol=1e-13)
+
+
+# ------------------------------------------------------------- fake-quant forward GEMM
+def _golden_fq():
+    rows = []
+    for ln in open(os.path.join(GOLDEN, "fq_gemm_operand.txt")).read().splitlines():
+        if ln.strip() and not ln.startswith("#"):
+            rows.append([float.fromhex(v) for v in ln.split()])
+    return rows
+
+
+def test_fq_gemm_golden_bf16_operand(oracle_mod):
+    """Hand-worked bf16 roundings of Q (ties to even, clamp, zero group): one weight per row,
+    x = 2 on that column, so Y = 2 * Qb exactly."""
+    rows = _golden_fq()
+    R, C = len(rows), 32
+    W = np.zeros((R, C), np.float32)
+    D = np.zeros((R, 1), np.float32)
+    for r, (w, d, _) in enumerate(rows):
+        W[r, r % C] = w
+        D[r, 0] = d
+    X = np.zeros((1, C), np.float32)
+    X[0, :R] = 2.0
+    Y = oracle_mod.fq_gemm(inputs.f32_to_bf16_bits(X), W, D)
+    np.testing.assert_array_equal(Y[0], [2.0 * e for _, _, e in rows])
+
+
+def test_fq_gemm_equals_export_product_on_exact_grids(oracle_mod):
+    """With power-of-two scales, fl(Delta*q) is a bf16 and a binary16 value, so the fake-quant
+    forward and the W4A16 product of the packed export are the same sum in the same order:
+    bitwise equal, although one goes through the LSQ forward and the other through packing and
+    nibble decoding."""
+    rng = np.random.default_rng(11)
+    T, R, C = 3, 7, 96
+    D = (2.0 ** -rng.integers(4, 9, (R, C // 32))).astype(np.float32)
+    W = (rng.standard_normal((R, C)) * 0.1).astype(np.float32)
+    Xb = inputs.f32_to_bf16_bits(rng.standard_normal((T, C)).astype(np.float32))
+    Y = oracle_mod.fq_gemm(Xb, W, D)
+    packed, scales = oracle_mod.pack_w4a16(W, D)
+    Yg = oracle_mod.w4a16_gemv(Xb, packed, scales, 32)
+    np.testing.assert_array_equal(Y, Yg)
+    assert np.count_nonzero(Y) == Y.size
+
+
+def test_fq_gemm_twin_and_entries(oracle_mod):
+    """The C oracle against the NumPy twin (own fake-quant, own bf16 rounding, BLAS product), and
+    its sampled-entry form against the full product (same sum order: bitwise)."""
+    rng = np.random.default_rng(12)
+    T, R, C = 5, 9, 64
+    W = (rng.standard_normal((R, C)) * 0.05).astype(np.float32)
+    D = (np.abs(W).reshape(R, C // 32, 32).max(axis=2) / 7 * rng.uniform(0.5, 1.0, (R, C // 32))).astype(np.float32)
+    Xb = inputs.f32_to_bf16_bits(rng.standard_normal((T, C)).astype(np.float32))
+    Y = oracle_mod.fq_gemm(Xb, W, D)
+    Yt = twin.fq_gemm(inputs.bf16_bits_to_f32(Xb), W, D)
+    np.testing.assert_allclose(Y, Yt, rtol=1e-12, atol=1e-15)
+    tt = rng.integers(0, T, 20)
+    rr = rng.integers(0, R, 20)
+    np.testing.assert_array_equal(oracle_mod.fq_gemm_entries(Xb, W, D, tt, rr), Y[tt, rr])
