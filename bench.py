@@ -667,6 +667,81 @@ def run_w4a16_decode(args):
         "stages": {f"M={M}": v for M, v in results.items()}}), flush=True)
 
 
+def run_fq_gemm(args):
+    """The fused fake-quant forward GEMM of a QAT step on the 1B-class up-projection (W fp32
+    8192x2048, searched-range scales) for a micro-batch of --tokens tokens: TFLOP/s against the
+    bf16 tensor peak, each launch timed with CUDA events after an L2 flush.  For context the
+    same product is also timed unfused through libraries: the LSQ forward, a cast to bf16 and a
+    cuBLAS bf16 GEMM."""
+    import torch
+
+    import int4_group_wise_b200 as q4
+    from int4_group_wise_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_kind = load_peaks()
+    wl = inputs.workload(1)
+    m = wl.matrices[0]
+    W_h = wl.weight(m)
+    R, C = W_h.shape
+    T = args.tokens
+    rng = np.random.default_rng(1)
+    D_h = (np.abs(W_h).reshape(R, C // 32, 32).max(axis=2) / np.float32(7) *
+           rng.uniform(0.5, 1.0, (R, C // 32))).astype(np.float32)
+    X = torch.from_numpy(wl.activations(m.x_name, n=T).view(np.int16)).to(dev).view(torch.bfloat16)
+    W = torch.from_numpy(W_h).to(dev)
+    D = torch.from_numpy(D_h).to(dev)
+    Y = torch.empty((T, R), dtype=torch.float32, device=dev)
+    Q = torch.empty_like(W)
+    flush_buf = torch.ones(128 << 20, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn, n):
+        ts = []
+        for _ in range(n):
+            torch.sum(flush_buf, dim=0, out=sink)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            ts.append((a, b))
+        torch.cuda.synchronize()
+        return sorted(a.elapsed_time(b) for a, b in ts)
+
+    fused = lambda: q4.fq_gemm(X, W, D, Y)
+
+    def unfused():
+        q4.lsq_fwd(W, D, Q)
+        torch.matmul(X, Q.to(torch.bfloat16).t())
+
+    for _ in range(args.warmup):
+        fused()
+        unfused()
+    q4.sync_check()
+    with ClockSampler(0) as clk:
+        t_f = timed(fused, args.steps)
+    t_u = timed(unfused, max(3, args.steps // 2))
+    q4.sync_check()
+    flop = 2.0 * T * R * C
+    ms = statistics.median(t_f)
+    tf = flop / ms / 1e9
+    peak = float(peaks["bf16_tflops"])
+    print(json.dumps({
+        "metric": "fused fake-quant GEMM TFLOP/s (Y = X bf16(Q_Delta(W))^T)", "value": tf, "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "variant": "fq-gemm", "data": "synthetic", "dtype": "bf16 x bf16 -> f32 (quantizer f32)",
+        "config": {"workload": f"1B-class up-projection W fp32 {R}x{C}, X bf16 {T}x{C} (micro-batch of {T} tokens)",
+                   "l2": "flushed (512 MB read sweep) before every launch"},
+        "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                     "flop_per_launch": flop, "peak_kind": f"{peak_kind} bf16 burst"},
+        "ms_min_median_max": [t_f[0], ms, t_f[-1]],
+        "unfused_library_ms": statistics.median(t_u),
+        "unfused_library": "qat4_lsq_fwd + cast to bf16 + torch.matmul (cuBLAS bf16), same product",
+        "gpu_launches": args.steps, "clocks": clk.summary()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -675,9 +750,11 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--variant", choices=["group32", "per-channel", "w4a16-decode"], default="group32",
+    ap.add_argument("--variant", choices=["group32", "per-channel", "w4a16-decode", "fq-gemm"], default="group32",
                     help="per-channel: time the one-scale-per-row LSQ step and export instead; "
-                         "w4a16-decode: time the inference GEMV on the packed 8B-class stack")
+                         "w4a16-decode: time the inference GEMV on the packed 8B-class stack; "
+                         "fq-gemm: time the fused fake-quant forward GEMM")
+    ap.add_argument("--tokens", type=int, default=8192, help="fq-gemm: tokens of the micro-batch")
     ap.add_argument("--layers", type=int, default=None,
                     help="w4a16-decode: number of layers of the 8B-class stack (default: all 32)")
     args = ap.parse_args()
@@ -689,6 +766,8 @@ def main():
         run_per_channel(args)
     elif args.variant == "w4a16-decode":
         run_w4a16_decode(args)
+    elif args.variant == "fq-gemm":
+        run_fq_gemm(args)
     else:
         run_ours(args)
 

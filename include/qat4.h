@@ -252,6 +252,23 @@ qat4_status qat4_scale_search_rowwise(const float *W, int64_t R, int64_t C,
 qat4_status qat4_w4a16_gemv(const uint16_t *x, int64_t M, const uint8_t *packed, const uint16_t *scales,
                             int64_t R, int64_t C, int64_t group, float *y, cudaStream_t stream);
 
+/* ------------------------------------------------ fake-quant forward GEMM
+ * The forward of a quantized linear layer in a QAT step (blog "Opt.Gear-QAT",
+ * section 3 "LSQ-based QAT": the forward pass runs on the weights projected
+ * onto the deployment INT4 grid), with the quantizer fused into the GEMM:
+ *     Y[t, r] = sum_c X[t, c] * bf16(Q_Delta(W)[r, c])
+ *  X      bf16 bit patterns [T, C], row-major (T tokens).
+ *  W      float32 [R, C], delta float32 [R, C/32]: Q_Delta(w) = Delta *
+ *         clamp(rint(w / Delta), -8, 7) exactly as qat4_lsq_fwd computes it,
+ *         then rounded to bf16 to nearest even (the operand precision of a bf16
+ *         forward); products exact, sums float32 on the tensor cores.
+ *  Y      out float32 [T, R], row-major.
+ *  C must be a multiple of 32; T, R >= 1.  Pointers 16-byte aligned.
+ *  Errors: QAT4_ERR_NULL, _SHAPE, _ALIGN, _CUDA; a bounded wait that gives up
+ *  leaves QAT4_ERR_TIMEOUT for qat4_sync_check. */
+qat4_status qat4_fq_gemm(const uint16_t *X, int64_t T, const float *W, const float *delta, int64_t R, int64_t C,
+                         float *Y, cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the library's device error
  * word for the current device.  Returns QAT4_ERR_TIMEOUT if a kernel gave up
  * a bounded wait since the last check, QAT4_ERR_CUDA if synchronisation

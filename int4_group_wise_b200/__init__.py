@@ -47,6 +47,7 @@ EXPORTS = {
     "qat4_scale_search_rowwise_workspace_bytes": (_Z, [_I64, _I64]),
     "qat4_scale_search_rowwise": (ct.c_int, [_P, _I64, _I64, _P, _I64, _P, _I32, _P, _P, _P, _P, _Z, _P]),
     "qat4_w4a16_gemv": (ct.c_int, [_P, _I64, _P, _P, _I64, _I64, _I64, _P, _P]),
+    "qat4_fq_gemm": (ct.c_int, [_P, _I64, _P, _P, _I64, _I64, _P, _P]),
     "qat4_sync_check": (ct.c_int, [_P]),
     "qat4_selftest_bounded_wait": (ct.c_int, [_I64, _P]),
 }
@@ -346,6 +347,24 @@ def w4a16_gemv(x, packed, scales, y=None, stream=None):
     _check(L.qat4_w4a16_gemv(_dev(x, "x"), M, _dev(packed, "packed"), _dev(scales, "scales"), R, C, C // G,
                              _dev(y, "y"), _stream(stream)), "qat4_w4a16_gemv")
     return y
+
+
+def fq_gemm(X, W, delta, Y=None, stream=None):
+    """Y [T, R] float32 = X @ bf16(Q_delta(W))^T; X bf16 [T, C], W float32 [R, C], delta float32
+    [R, C/32]."""
+    import torch
+    L = lib()
+    _dev(X, "X", torch.bfloat16)
+    T, C = X.shape
+    _dev(W, "W", torch.float32)
+    R = W.shape[0]
+    if W.shape[1] != C:
+        raise ValueError("W must be [R, C] with the C of X")
+    _dev(delta, "delta", torch.float32, (R, C // 32))
+    Y = _out(Y, "Y", (T, R), torch.float32, X)
+    _check(L.qat4_fq_gemm(_dev(X, "X"), T, _dev(W, "W"), _dev(delta, "delta"), R, C, _dev(Y, "Y"),
+                          _stream(stream)), "qat4_fq_gemm")
+    return Y
 
 
 def sync_check(stream=None):

@@ -20,6 +20,7 @@
 #include "rowwise.cuh"
 #include "rowwise_search.cuh"
 #include "w4a16_gemv.cuh"
+#include "fq_gemm.cuh"
 
 namespace {
 
@@ -38,6 +39,7 @@ struct DeviceInfo {
     bool search_attr = false;
     bool rowsearch_attr = false;
     int smem_optin = 0;       // opt-in shared memory per block; gemv attributes set when > 0
+    bool fq_attr = false;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mutex;
@@ -474,6 +476,66 @@ qat4_status qat4_w4a16_gemv(const uint16_t* x, int64_t M, const uint8_t* packed,
         if (cudaGetLastError() != cudaSuccess) return QAT4_ERR_CUDA;
     }
     return QAT4_OK;
+}
+
+// ------------------------------------------------------ fake-quant forward GEMM
+qat4_status qat4_fq_gemm(const uint16_t* X, int64_t T, const float* W, const float* delta, int64_t R, int64_t C,
+                         float* Y, cudaStream_t stream) {
+    if (!X || !W || !delta || !Y) return QAT4_ERR_NULL;
+    if (T < 1 || T > (int64_t(1) << 31) - 1 || !valid_rc(R, C) || T * R > (int64_t(1) << 40)) return QAT4_ERR_SHAPE;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(delta) || !aligned16(Y)) return QAT4_ERR_ALIGN;
+    const int64_t tiles_m = (T + qat4::kFqTile * qat4::kFqMTiles - 1) / (qat4::kFqTile * qat4::kFqMTiles);
+    const int64_t tiles_r = (R + qat4::kFqTile - 1) / qat4::kFqTile;
+    if (2 * tiles_m * tiles_r > (int64_t(1) << 31) - 1) return QAT4_ERR_SHAPE;
+    int dev = 0;
+    DeviceInfo* info = nullptr;
+    if (!device_info(&dev, &info)) return QAT4_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!info->fq_attr) {
+            if (cudaFuncSetAttribute(qat4::fq_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(qat4::kFqSmemBytes)) != cudaSuccess)
+                return QAT4_ERR_CUDA;
+            info->fq_attr = true;
+        }
+    }
+    EncodeTiledFn encode = encode_tiled();
+    if (!encode) return QAT4_ERR_CUDA;
+    CUtensorMap tx, tw;
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(T)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(C) * 2};
+        const cuuint32_t box[2] = {static_cast<cuuint32_t>(qat4::kFqBK), static_cast<cuuint32_t>(qat4::kFqHalf)};
+        const cuuint32_t estr[2] = {1, 1};
+        if (encode(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return QAT4_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(R)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(C) * 4};
+        const cuuint32_t box[2] = {32, static_cast<cuuint32_t>(qat4::kFqHalf)};
+        const cuuint32_t estr[2] = {1, 1};
+        if (encode(&tw, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(W), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return QAT4_ERR_CUDA;
+    }
+    qat4::FqParams p;
+    p.delta = delta;
+    p.Y = Y;
+    p.T = static_cast<int>(T);
+    p.R = static_cast<int>(R);
+    p.C = static_cast<int>(C);
+    p.G = static_cast<int>(C / 32);
+    p.tiles_r = static_cast<int>(tiles_r);
+    p.ksteps = static_cast<int>((C + qat4::kFqBK - 1) / qat4::kFqBK);
+    // generous bound: 4 s plus 10 us per 64-column step (a step takes well under 1 us)
+    p.limit_ns = 4000000000ull + 10000ull * static_cast<uint64_t>(p.ksteps);
+    const unsigned grid = static_cast<unsigned>(2 * tiles_m * tiles_r);
+    qat4::fq_gemm_kernel<<<grid, qat4::kFqThreads, qat4::kFqSmemBytes, stream>>>(tx, tw, p);
+    return launch_status();
 }
 
 // ------------------------------------------------------------ error handling

@@ -254,8 +254,6 @@ w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tmap, const GemvParams p) 
         uint4 wq[RPW];
 #pragma unroll
         for (int r = 0; r < RPW; ++r) wq[r] = *reinterpret_cast<const uint4*>(st + r * kGvRowBytes);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[s]);
         const int bn = ch + 1 == nchunks ? b + 1 : b, chn = ch + 1 == nchunks ? 0 : ch + 1;
         if (t + 1 < t1) gv_scales<RPW>(p.scales, R, G, C, group, bn, chn, row0, lane, s_next);
 
@@ -306,6 +304,11 @@ w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tmap, const GemvParams p) 
 #pragma unroll
                 for (int m = 0; m < MT; ++m) acc[r][m] = fmaf(s_cur[r], part[r][m].x + part[r][m].y, acc[r][m]);
         }
+        // the slot is released only once the codes loaded from it have been used: a release
+        // issued while a shared load is still in flight does not keep the next bulk copy from
+        // overwriting the slot under it
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty_bar[s]);
 
         if (ch == nchunks - 1 || t == t1 - 1) {
 #pragma unroll

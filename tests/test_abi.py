@@ -99,3 +99,13 @@ def test_pack_search_hessian_validation():
 def test_w4a16_gemv_validation(args, code):
     x, M, packed, scales, R, C, group, y = args
     assert q4.lib().qat4_w4a16_gemv(x, M, packed, scales, R, C, group, y, None) == code
+
+
+def test_fq_gemm_validation():
+    L = q4.lib()
+    assert L.qat4_fq_gemm(None, 8, A, A, 8, 64, A, None) == 1
+    assert L.qat4_fq_gemm(A, 0, A, A, 8, 64, A, None) == 2
+    assert L.qat4_fq_gemm(A, 8, A, A, 8, 48, A, None) == 2
+    assert L.qat4_fq_gemm(A, 8, A, A, 0, 64, A, None) == 2
+    assert L.qat4_fq_gemm(A, 8, MIS, A, 8, 64, A, None) == 3
+    assert L.qat4_fq_gemm(A, 8, A, A, 8, 64, MIS, None) == 3

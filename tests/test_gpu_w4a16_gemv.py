@@ -61,3 +61,17 @@ def test_gemv_layer_shape(oracle_mod):
     W, D = _export(14336, 4096, seed=5)
     for M in (1, 4):
         _check(W, D, M, oracle_mod)
+
+
+def test_gemv_deterministic():
+    """Repeated launches give bitwise identical y (two partial sums per cut row block at most,
+    and no ring slot is refilled before its codes are used)."""
+    W, D = _export(14336, 4096, seed=6)
+    packed, scales = q4.pack_w4a16(torch.from_numpy(W).cuda(), torch.from_numpy(D).cuda())
+    for M in (1, 4):
+        xb = inputs.activations(M, 4096, seed=M, cfg=91, name="xdet", outliers=40)
+        tx = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+        y0 = q4.w4a16_gemv(tx, packed, scales).clone()
+        for _ in range(30):
+            assert torch.equal(q4.w4a16_gemv(tx, packed, scales), y0)
+    q4.sync_check()
