@@ -742,6 +742,80 @@ def run_fq_gemm(args):
         "gpu_launches": args.steps, "clocks": clk.summary()}), flush=True)
 
 
+def run_hessian_split(args):
+    """The Hessian of the 1B-class up-projection's calibration set (X bf16 262144x2048) with its
+    rows split across the N ranks: each rank computes the partial of its shard on the tensor
+    cores, then one NCCL all-reduce sums the partials (16.8 MB).  Total work is fixed as N grows
+    (strong scaling); the time of a step is the slowest rank's, measured with CUDA events around
+    partial + all-reduce, L2 flushed before each step."""
+    from datetime import timedelta
+
+    import torch
+    import torch.distributed as dist
+
+    import int4_group_wise_b200 as q4
+    from int4_group_wise_b200 import distributed, inputs
+
+    rank, world, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world == 1:   # a one-rank group still runs the all-reduce path
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", "29533")
+    dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev, rank=rank, world_size=world)
+    try:
+        peaks, peak_kind = load_peaks()
+        wl = inputs.workload(1)
+        m = wl.matrices[0]
+        n, C = wl.n_calib, wl.calib[m.x_name]
+        lo, hi = distributed.shard_rows(n, world, rank)
+        Xb = wl.activations(m.x_name)[lo:hi]
+        X = torch.from_numpy(np.ascontiguousarray(Xb).view(np.int16)).to(dev).view(torch.bfloat16)
+        del Xb
+        H = torch.empty((C, C), dtype=torch.float32, device=dev)
+        ws = torch.empty(max(1, q4.hessian_workspace_bytes(hi - lo, C)), dtype=torch.uint8, device=dev)
+        flush_buf = torch.ones(128 << 20, dtype=torch.float32, device=dev)
+        sink = torch.empty((), dtype=torch.float32, device=dev)
+        stream = torch.cuda.current_stream(dev)
+        step = lambda: distributed.hessian_sharded(X, n, H=H, workspace=ws)
+        for _ in range(args.warmup):
+            step()
+        torch.cuda.synchronize()
+        q4.sync_check()
+        ts = []
+        with ClockSampler(local) as clk:
+            for _ in range(args.steps):
+                torch.sum(flush_buf, dim=0, out=sink)
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                dist.barrier()
+                a.record(stream)
+                step()
+                b.record(stream)
+                ts.append((a, b))
+            torch.cuda.synchronize()
+        q4.sync_check()
+        ms_local = statistics.median(a.elapsed_time(b) for a, b in ts)
+        _, ms = aggregate_over_ranks(0.0, ms_local)
+        flop = float(n) * C * (C + 1)
+        tf = flop / ms / 1e9
+        peak = float(peaks["bf16_tflops"]) * world
+        if rank == 0:
+            print(json.dumps({
+                "metric": "split-n Hessian TFLOP/s (partials + NCCL all-reduce)", "value": tf, "unit": "TFLOP/s",
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "strong", "variant": "hessian-split", "data": "synthetic",
+                "dtype": "bf16 x bf16 -> f32",
+                "config": {"workload": f"1B-class up-projection calibration set X bf16 {n}x{C}, rows split "
+                                       f"over {world} GPU(s)", "parallelism": f"split-n x{world} + all-reduce",
+                           "l2": "flushed (512 MB read sweep) before every step"},
+                "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
+                             "peak_kind": f"{peak_kind} bf16 burst x {world} GPU(s)"},
+                "allreduce_bytes": C * C * 4, "gpu_launches": args.steps * (1 if q4.hessian_workspace_bytes(
+                    hi - lo, C) == 0 else 2), "clocks": clk.summary()}), flush=True)
+    finally:
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -750,10 +824,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--variant", choices=["group32", "per-channel", "w4a16-decode", "fq-gemm"], default="group32",
+    ap.add_argument("--variant", choices=["group32", "per-channel", "w4a16-decode", "fq-gemm", "hessian-split"],
+                    default="group32",
                     help="per-channel: time the one-scale-per-row LSQ step and export instead; "
                          "w4a16-decode: time the inference GEMV on the packed 8B-class stack; "
-                         "fq-gemm: time the fused fake-quant forward GEMM")
+                         "fq-gemm: time the fused fake-quant forward GEMM; "
+                         "hessian-split: the calibration Hessian with its rows split over the ranks")
     ap.add_argument("--tokens", type=int, default=8192, help="fq-gemm: tokens of the micro-batch")
     ap.add_argument("--layers", type=int, default=None,
                     help="w4a16-decode: number of layers of the 8B-class stack (default: all 32)")
@@ -768,6 +844,8 @@ def main():
         run_w4a16_decode(args)
     elif args.variant == "fq-gemm":
         run_fq_gemm(args)
+    elif args.variant == "hessian-split":
+        run_hessian_split(args)
     else:
         run_ours(args)
 

@@ -89,6 +89,14 @@ size_t qat4_hessian_workspace_bytes(int64_t n, int64_t C);
 qat4_status qat4_hessian(const uint16_t *X, int64_t n, int64_t C, float *H,
                          void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* One rank's share of a Hessian whose calibration rows are split across GPUs:
+ * H = X^T X / n_total over the n rows of X (n <= n_total), everything else as
+ * qat4_hessian (same workspace size for the same n and C).  Summing the
+ * partials of all shards (an all-reduce) gives X_all^T X_all / n_total:
+ * the split-n form of the exchange step of the Hessian on several GPUs. */
+qat4_status qat4_hessian_partial(const uint16_t *X, int64_t n, int64_t C, int64_t n_total, float *H,
+                                 void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* ---------------------------------------------------------------- (b)
  * Hessian-weighted per-group scale search (model card, "Quantization
  * Configuration": Delta* = argmin ||W X - Q_Delta(W) X||_F^2 per group,

@@ -34,6 +34,7 @@ EXPORTS = {
     "qat4_abi_version": (ct.c_int, []),
     "qat4_hessian_workspace_bytes": (_Z, [_I64, _I64]),
     "qat4_hessian": (ct.c_int, [_P, _I64, _I64, _P, _P, _Z, _P]),
+    "qat4_hessian_partial": (ct.c_int, [_P, _I64, _I64, _I64, _P, _P, _Z, _P]),
     "qat4_hessian_noalloc": (ct.c_int, [_P, _I64, _I64, _P, _P]),
     "qat4_scale_search": (ct.c_int, [_P, _I64, _I64, _P, _I64, _P, _I32, _P, _P, _P, _P]),
     "qat4_lsq_fwd": (ct.c_int, [_P, _P, _I64, _I64, _P, _P]),
@@ -131,6 +132,24 @@ def hessian(X, H=None, workspace=None, stream=None):
     wp = _dev(workspace, "workspace", torch.uint8) if workspace is not None else None
     wbytes = workspace.numel() if workspace is not None else 0
     _check(L.qat4_hessian(_dev(X, "X"), n, C, _dev(H, "H"), wp, wbytes, _stream(stream)), "qat4_hessian")
+    return H
+
+
+def hessian_partial(X, n_total, H=None, workspace=None, stream=None):
+    """One shard's share of a split-n Hessian: H = X^T X / n_total for this shard's rows X bf16
+    [n, C]; the sum of all shards' partials is the Hessian of all n_total rows."""
+    import torch
+    L = lib()
+    _dev(X, "X", torch.bfloat16)
+    n, C = X.shape
+    H = _out(H, "H", (C, C), torch.float32, X)
+    need = hessian_workspace_bytes(n, C)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    wp = _dev(workspace, "workspace", torch.uint8) if workspace is not None else None
+    wbytes = workspace.numel() if workspace is not None else 0
+    _check(L.qat4_hessian_partial(_dev(X, "X"), n, C, int(n_total), _dev(H, "H"), wp, wbytes, _stream(stream)),
+           "qat4_hessian_partial")
     return H
 
 

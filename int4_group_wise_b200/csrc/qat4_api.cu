@@ -122,10 +122,16 @@ size_t qat4_hessian_workspace_bytes(int64_t n, int64_t C) {
     return static_cast<size_t>(plan.tiles) * plan.split * qat4::kPTile * qat4::kPTile * sizeof(float);
 }
 
-qat4_status qat4_hessian(const uint16_t* X, int64_t n, int64_t C, float* H,
-                         void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// H = X^T X / n_norm over the n rows of X (n_norm = n for the Hessian itself).
+qat4_status hessian_run(const uint16_t* X, int64_t n, int64_t C, int64_t n_norm, float* H, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream) {
     if (!X || !H) return QAT4_ERR_NULL;
-    if (n < 1 || n > (int64_t(1) << 31) - 1 || C < 32 || C % 32 != 0 || C > 65536) return QAT4_ERR_SHAPE;
+    if (n < 1 || n > (int64_t(1) << 31) - 1 || C < 32 || C % 32 != 0 || C > 65536 || n_norm < 1)
+        return QAT4_ERR_SHAPE;
     if (!aligned16(X) || !aligned16(H) || (workspace && !aligned16(workspace))) return QAT4_ERR_ALIGN;
     const size_t need = qat4_hessian_workspace_bytes(n, C);
     if (workspace_bytes < need || (need > 0 && !workspace)) return QAT4_ERR_WORKSPACE;
@@ -159,7 +165,7 @@ qat4_status qat4_hessian(const uint16_t* X, int64_t n, int64_t C, float* H,
     p.n = n;
     p.C = static_cast<int>(C);
     p.plan = qat4::hess_plan(n, C);
-    p.inv_n = static_cast<float>(1.0 / static_cast<double>(n));
+    p.inv_n = static_cast<float>(1.0 / static_cast<double>(n_norm));
     // generous bound: 4 s plus 100 ns per calibration row (a chunk of the
     // mainloop takes ~2 ns per row at full rate)
     p.limit_ns = 4000000000ull + 100ull * static_cast<uint64_t>(n);
@@ -172,6 +178,21 @@ qat4_status qat4_hessian(const uint16_t* X, int64_t n, int64_t C, float* H,
         qat4::hessian_reduce_kernel<<<grid, 256, 0, stream>>>(static_cast<const float*>(workspace), p, H);
     }
     return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+qat4_status qat4_hessian(const uint16_t* X, int64_t n, int64_t C, float* H,
+                         void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    return hessian_run(X, n, C, n, H, workspace, workspace_bytes, stream);
+}
+
+qat4_status qat4_hessian_partial(const uint16_t* X, int64_t n, int64_t C, int64_t n_total, float* H,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (n_total < n) return QAT4_ERR_SHAPE;
+    return hessian_run(X, n, C, n_total, H, workspace, workspace_bytes, stream);
 }
 
 // -------------------------------------------------------------- scale search

@@ -109,3 +109,11 @@ def test_fq_gemm_validation():
     assert L.qat4_fq_gemm(A, 8, A, A, 0, 64, A, None) == 2
     assert L.qat4_fq_gemm(A, 8, MIS, A, 8, 64, A, None) == 3
     assert L.qat4_fq_gemm(A, 8, A, A, 8, 64, MIS, None) == 3
+
+
+def test_hessian_partial_validation():
+    L = q4.lib()
+    assert L.qat4_hessian_partial(None, 64, 64, 64, A, None, 0, None) == 1
+    assert L.qat4_hessian_partial(A, 64, 64, 63, A, None, 0, None) == 2      # n_total < n
+    assert L.qat4_hessian_partial(A, 64, 40, 64, A, None, 0, None) == 2
+    assert L.qat4_hessian_partial(MIS, 64, 64, 128, A, None, 0, None) == 3

@@ -128,3 +128,48 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     q4.sync_check()                                        # cleared
     Xb = inputs.activations(64, 64, seed=1, cfg=61, name="X")
     _gpu_h(Xb)                                             # kernels still run afterwards
+
+
+def test_split_n_partials_sum_to_the_hessian(oracle_mod):
+    """The split-n exchange step: partials X_r^T X_r / n over 4 ragged row shards (one of them
+    spanning several promotion chunks) add up to H within the same bound; small-integer X makes
+    every partial and their sum exact, so there it is bitwise."""
+    from int4_group_wise_b200 import distributed
+    n, C = 40000, 256
+    Xb = inputs.activations(n, C, seed=21, cfg=60, name="Xsplit", outliers=3)
+    X = torch.from_numpy(Xb.view(np.int16)).cuda().view(torch.bfloat16)
+    parts = [q4.hessian_partial(X[lo:hi], n) for lo, hi in (distributed.shard_rows(n, 4, r) for r in range(4))]
+    q4.sync_check()
+    Hs = sum(p.double() for p in parts).cpu().numpy()
+    assert _frob(Hs, oracle_mod.hessian(Xb)) <= 1e-3
+    # exact case: integer-valued X and n a power of two (1/n exact)
+    rng = np.random.default_rng(5)
+    Xi = inputs.f32_to_bf16_bits(rng.integers(-3, 4, (4096, 64)).astype(np.float32))
+    Xt = torch.from_numpy(Xi.view(np.int16)).cuda().view(torch.bfloat16)
+    Hfull = q4.hessian(Xt)
+    Hsum = q4.hessian_partial(Xt[:1000], 4096) + q4.hessian_partial(Xt[1000:], 4096)
+    q4.sync_check()
+    assert torch.equal(Hsum, Hfull)
+
+
+def test_hessian_sharded_single_rank_nccl():
+    """hessian_sharded end to end (partial on the tensor cores, then the NCCL all-reduce) in a
+    one-rank process group: the all-reduce is the identity, so H equals qat4_hessian's."""
+    import os
+    import socket
+    import torch.distributed as dist
+    from int4_group_wise_b200 import distributed
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("nccl", rank=0, world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        Xb = inputs.activations(3000, 512, seed=2, cfg=60, name="Xnccl", outliers=5)
+        X = torch.from_numpy(Xb.view(np.int16)).cuda().view(torch.bfloat16)
+        H = distributed.hessian_sharded(X, 3000)
+        torch.cuda.synchronize()
+        q4.sync_check()
+        assert torch.equal(H, q4.hessian(X))
+    finally:
+        dist.destroy_process_group()

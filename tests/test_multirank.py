@@ -61,3 +61,65 @@ def test_reference_arm_prints_only_on_rank0(tmp_path):
                         "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True,
                        timeout=300, cwd=ROOT)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+# ------------------------------------------------------------- split-n Hessian plumbing
+def _hessian_worker(rank, world, port, n, C, out):
+    """Each rank takes its shard of the calibration rows, forms its partial X_r^T X_r / n with
+    the oracle (CPU stand-in for the kernel's qat4_hessian_partial), and the all-reduce of the
+    distributed module sums them."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import oracle
+    from int4_group_wise_b200 import distributed, inputs
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        Xb = inputs.activations(n, C, seed=3, cfg=0, name="split", outliers=2)
+        lo, hi = distributed.shard_rows(n, world, rank)
+        part = oracle.hessian(Xb[lo:hi]) * ((hi - lo) / n)
+        H = torch.from_numpy(part.astype(np.float32))
+        distributed.allreduce_partials(H)
+        out.put((rank, lo, hi, H.numpy()))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_split_n_hessian_allreduce_two_gloo_ranks():
+    import numpy as np
+    sys.path.insert(0, ROOT)
+    import oracle
+    from int4_group_wise_b200 import inputs
+    n, C = 1001, 64
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_hessian_worker, args=(r, 2, port, n, C, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted((q.get(timeout=180) for _ in procs), key=lambda t: t[0])
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    # the shards tile [0, n) exactly, and both ranks hold the same, full H
+    assert [(lo, hi) for _, lo, hi, _ in res] == [(0, 500), (500, 1001)]
+    np.testing.assert_array_equal(res[0][3], res[1][3])
+    Href = oracle.hessian(inputs.activations(n, C, seed=3, cfg=0, name="split", outliers=2))
+    np.testing.assert_allclose(res[0][3], Href, rtol=1e-6, atol=1e-6 * np.abs(Href).max())
+
+
+def test_shard_rows_partition():
+    sys.path.insert(0, ROOT)
+    from int4_group_wise_b200 import distributed
+    for n in (1, 7, 64, 262144, 1000003):
+        for world in (1, 2, 3, 4, 8):
+            bounds = [distributed.shard_rows(n, world, r) for r in range(world)]
+            assert bounds[0][0] == 0 and bounds[-1][1] == n
+            assert all(bounds[r][1] == bounds[r + 1][0] for r in range(world - 1))
+            sizes = [hi - lo for lo, hi in bounds]
+            assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(ValueError):
+        distributed.shard_rows(10, 2, 2)
