@@ -235,3 +235,34 @@ def fq_gemm_entries(X_bits: np.ndarray, W: np.ndarray, delta: np.ndarray, tt, rr
     out = np.empty(tt.size, np.float64)
     lib().oracle_fq_gemm_entries(_p(X), _p(W), _p(delta), X.shape[1], tt.size, _p(tt), _p(rr), _p(out))
     return out
+
+
+def refine(W: np.ndarray, H: np.ndarray, alpha: np.ndarray, idx_start: np.ndarray, sweeps: int = 1):
+    """Full-objective coordinate descent from idx_start: (delta float32 [R, G], idx int32 [R, G],
+    obj float64 [R])."""
+    W = _c(W, np.float32)
+    H = _c(H, np.float32)
+    alpha = _c(alpha, np.float32)
+    R, C = W.shape
+    idx = _c(idx_start, np.int32).copy()
+    delta = np.empty((R, C // 32), np.float32)
+    obj = np.empty(R, np.float64)
+    lib().oracle_refine(_p(W), R, C, _p(H), H.shape[1], _p(alpha), alpha.size, int(sweeps), _p(idx),
+                        _p(delta), _p(obj))
+    return delta, idx, obj
+
+
+def refine_replay(W: np.ndarray, H: np.ndarray, alpha: np.ndarray, idx_start: np.ndarray, idx_pick: np.ndarray):
+    """For one sweep that moved idx_start to idx_pick: per (row, group) the minimum of the full
+    objective over the group's candidates at that point of the sweep, and its value at the pick."""
+    W = _c(W, np.float32)
+    H = _c(H, np.float32)
+    alpha = _c(alpha, np.float32)
+    R, C = W.shape
+    s = _c(idx_start, np.int32)
+    k = _c(idx_pick, np.int32)
+    emin = np.empty((R, C // 32), np.float64)
+    epick = np.empty((R, C // 32), np.float64)
+    lib().oracle_refine_replay(_p(W), R, C, _p(H), H.shape[1], _p(alpha), alpha.size, _p(s), _p(k), _p(emin),
+                               _p(epick))
+    return emin, epick

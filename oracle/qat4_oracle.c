@@ -503,3 +503,112 @@ void oracle_fq_gemm_entries(const uint16_t *X, const float *W, const float *delt
         out[m] = s;
     }
 }
+
+/* -------------------------------------------- full-objective refinement
+ * The model card ("Quantization Configuration") writes the objective over the
+ * whole layer, Delta* = argmin ||W X - Q_Delta(W) X||_F^2, i.e. per row of W
+ * the quadratic form e H e^T of e = w - Q_Delta(w) over all C columns.  The
+ * search above keeps only the diagonal 32x32 blocks of H (each group on its
+ * own).  This refinement starts from given candidate indices (the search's)
+ * and runs `sweeps` passes of coordinate descent: groups in order g = 0..G-1,
+ * each set to the candidate of its own grid (Delta_k = alpha_k * fl(m/7), as in
+ * the search) that minimises the full objective with every other group held
+ * at its current scale; ties go to the smallest k.  Every candidate's
+ * objective is evaluated in full (all C x C terms, binary64, e exact).
+ * W: float [R, C]; H: float, row stride ldh; alpha [K];
+ * idx_io: int32 [R, C/32], start indices in, refined indices out;
+ * delta_out: float [R, C/32]; obj_out: double [R], final objective. */
+static double full_objective(const double *e, const float *H, int64_t ldh, int64_t C)
+{
+    double E = 0.0;
+    for (int64_t i = 0; i < C; ++i) {
+        double row = 0.0;
+        for (int64_t j = 0; j < C; ++j) row += (double)H[i * ldh + j] * e[j];
+        E += e[i] * row;
+    }
+    return E;
+}
+
+static void group_error(const float *w, float dk, double *e)
+{
+    for (int i = 0; i < GROUP; ++i) e[i] = (double)w[i] - (double)fake_quant(w[i], dk);
+}
+
+static float group_base(const float *w)
+{
+    float m = 0.0f;
+    for (int i = 0; i < GROUP; ++i) {
+        float a = fabsf(w[i]);
+        if (a > m) m = a;
+    }
+    return m / 7.0f;
+}
+
+void oracle_refine(const float *W, int64_t R, int64_t C, const float *H, int64_t ldh,
+                   const float *alpha, int32_t K, int32_t sweeps,
+                   int32_t *idx_io, float *delta_out, double *obj_out)
+{
+    const int64_t G = C / GROUP;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < R; ++r) {
+        const float *w = W + r * C;
+        int32_t *idx = idx_io + r * G;
+        double *e = (double *)malloc((size_t)C * sizeof(double));
+        for (int64_t g = 0; g < G; ++g)
+            group_error(w + g * GROUP, alpha[idx[g]] * group_base(w + g * GROUP), e + g * GROUP);
+        for (int32_t s = 0; s < sweeps; ++s) {
+            for (int64_t g = 0; g < G; ++g) {
+                const float base = group_base(w + g * GROUP);
+                int32_t best_k = -1;
+                double best = 0.0;
+                for (int32_t k = 0; k < K; ++k) {
+                    group_error(w + g * GROUP, alpha[k] * base, e + g * GROUP);
+                    const double E = full_objective(e, H, ldh, C);
+                    if (best_k < 0 || E < best) {
+                        best = E;
+                        best_k = k;
+                    }
+                }
+                idx[g] = best_k;
+                group_error(w + g * GROUP, alpha[best_k] * base, e + g * GROUP);
+            }
+        }
+        for (int64_t g = 0; g < G; ++g) delta_out[r * G + g] = alpha[idx[g]] * group_base(w + g * GROUP);
+        obj_out[r] = full_objective(e, H, ldh, C);
+        free(e);
+    }
+}
+
+/* One sweep replayed with given choices, for checking another implementation's
+ * sweep: start from idx_start and, for g = 0..G-1 in order, evaluate every
+ * candidate of group g in full (other groups: idx_pick for groups < g,
+ * idx_start for groups > g), report the minimum (emin) and the objective at
+ * idx_pick[g] (epick), then move group g to idx_pick[g].  Outputs [R, C/32]. */
+void oracle_refine_replay(const float *W, int64_t R, int64_t C, const float *H, int64_t ldh,
+                          const float *alpha, int32_t K, const int32_t *idx_start,
+                          const int32_t *idx_pick, double *emin, double *epick)
+{
+    const int64_t G = C / GROUP;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < R; ++r) {
+        const float *w = W + r * C;
+        double *e = (double *)malloc((size_t)C * sizeof(double));
+        for (int64_t g = 0; g < G; ++g)
+            group_error(w + g * GROUP, alpha[idx_start[r * G + g]] * group_base(w + g * GROUP), e + g * GROUP);
+        for (int64_t g = 0; g < G; ++g) {
+            const float base = group_base(w + g * GROUP);
+            const int32_t pick = idx_pick[r * G + g];
+            double best = 0.0, at_pick = 0.0;
+            for (int32_t k = 0; k < K; ++k) {
+                group_error(w + g * GROUP, alpha[k] * base, e + g * GROUP);
+                const double E = full_objective(e, H, ldh, C);
+                if (k == 0 || E < best) best = E;
+                if (k == pick) at_pick = E;
+            }
+            emin[r * G + g] = best;
+            epick[r * G + g] = at_pick;
+            group_error(w + g * GROUP, alpha[pick] * base, e + g * GROUP);
+        }
+        free(e);
+    }
+}

@@ -95,3 +95,35 @@ def fq_gemm(X, W, delta):
     D = np.repeat(np.asarray(delta, f32), 32, axis=1)
     Qb = _bf16_rne(fake_quant(W, D)).astype(np.float64)
     return np.asarray(X, np.float64) @ Qb.T
+
+
+def refine(W, H, alpha, idx_start, sweeps):
+    """Coordinate descent on the full objective e H e^T (groups in order, ties to the smallest k),
+    every candidate's objective evaluated with a float64 matrix product."""
+    W = np.asarray(W, f32)
+    H = np.asarray(H, np.float64)
+    alpha = np.asarray(alpha, f32)
+    R, C = W.shape
+    G = C // 32
+    idx = np.array(idx_start, np.int32, copy=True)
+    obj = np.empty(R)
+    for r in range(R):
+        wg = W[r].reshape(G, 32)
+        base = (np.abs(wg).max(axis=1) / f32(7)).astype(f32)
+
+        def err(g, k):
+            return wg[g].astype(np.float64) - fake_quant(wg[g], (alpha[k] * base[g]).astype(f32)).astype(np.float64)
+
+        e = np.concatenate([err(g, idx[r, g]) for g in range(G)])
+        for _ in range(sweeps):
+            for g in range(G):
+                best_k, best = -1, 0.0
+                for k in range(alpha.size):
+                    e[32 * g:32 * g + 32] = err(g, k)
+                    E = float(e @ H @ e)
+                    if best_k < 0 or E < best:
+                        best_k, best = k, E
+                idx[r, g] = best_k
+                e[32 * g:32 * g + 32] = err(g, best_k)
+        obj[r] = float(e @ H @ e)
+    return idx, obj

@@ -586,3 +586,73 @@ def test_fq_gemm_twin_and_entries(oracle_mod):
     tt = rng.integers(0, T, 20)
     rr = rng.integers(0, R, 20)
     np.testing.assert_array_equal(oracle_mod.fq_gemm_entries(Xb, W, D, tt, rr), Y[tt, rr])
+
+
+# --------------------------------------------------------- full-objective refinement
+def _refine_problem(R, C, K, seed, coupled=True):
+    rng = np.random.default_rng(seed)
+    W = (rng.standard_normal((R, C)) * 0.02).astype(np.float32)
+    if coupled:
+        X = rng.standard_normal((4 * C, C)).astype(np.float32)
+        X[:, :C // 2] += X[:, C // 2:]                      # correlate channels across groups
+        H = (X.astype(np.float64).T @ X / X.shape[0]).astype(np.float32)
+    else:
+        H = np.zeros((C, C), np.float32)
+        for g in range(C // 32):
+            B = rng.standard_normal((64, 32))
+            H[32 * g:32 * g + 32, 32 * g:32 * g + 32] = (B.T @ B / 64).astype(np.float32)
+    alpha = inputs.alpha_grid(0.5, 0.5 / (K - 1), K)
+    return W, H, alpha
+
+
+def test_refine_keeps_the_search_when_H_is_block_diagonal(oracle_mod):
+    """Without cross-group blocks the full objective is the sum of the groups' own objectives,
+    which the search already minimises group by group: no sweep changes anything, and the final
+    objective is the sum of the search's per-group minima."""
+    W, H, alpha = _refine_problem(8, 128, 11, seed=31, coupled=False)
+    _, idx0, best, _ = oracle_mod.scale_search(W, H, alpha, all_err=True)
+    _, idx, obj = oracle_mod.refine(W, H, alpha, idx0, sweeps=3)
+    np.testing.assert_array_equal(idx, idx0)
+    np.testing.assert_allclose(obj, best.sum(axis=1), rtol=1e-12)
+
+
+def test_refine_agrees_with_twin(oracle_mod):
+    W, H, alpha = _refine_problem(5, 128, 9, seed=32)
+    _, idx0, _, _ = oracle_mod.scale_search(W, H, alpha, all_err=True)
+    _, idx, obj = oracle_mod.refine(W, H, alpha, idx0, sweeps=2)
+    idx_t, obj_t = twin.refine(W, H, alpha, idx0, 2)
+    np.testing.assert_array_equal(idx, idx_t)
+    np.testing.assert_allclose(obj, obj_t, rtol=1e-11)
+
+
+def test_refine_descends_to_a_coordinate_minimum(oracle_mod):
+    """From the search's scales, sweeps never raise the full objective, lower it where groups are
+    coupled, and stop at a point where no single group can improve it (checked by brute force
+    with the twin's objective)."""
+    W, H, alpha = _refine_problem(6, 96, 7, seed=33)
+    _, idx0, _, _ = oracle_mod.scale_search(W, H, alpha, all_err=True)
+    _, _, obj0 = oracle_mod.refine(W, H, alpha, idx0, sweeps=0)
+    _, idx, obj = oracle_mod.refine(W, H, alpha, idx0, sweeps=20)
+    assert np.all(obj <= obj0 * (1 + 1e-12))
+    assert np.any(obj < obj0 * (1 - 1e-6))
+    Hd = H.astype(np.float64)
+    for r in range(W.shape[0]):
+        wg = W[r].reshape(-1, 32)
+        base = (np.abs(wg).max(axis=1) / np.float32(7)).astype(np.float32)
+        err = lambda g, k: wg[g].astype(np.float64) - twin.fake_quant(wg[g], (alpha[k] * base[g]).astype(np.float32))
+        e = np.concatenate([err(g, idx[r, g]) for g in range(wg.shape[0])])
+        E = e @ Hd @ e
+        for g in range(wg.shape[0]):
+            for k in range(alpha.size):
+                e2 = e.copy()
+                e2[32 * g:32 * g + 32] = err(g, k)
+                assert e2 @ Hd @ e2 >= E * (1 - 1e-12)
+
+
+def test_refine_replay_of_its_own_sweep(oracle_mod):
+    W, H, alpha = _refine_problem(4, 128, 9, seed=34)
+    _, idx0, _, _ = oracle_mod.scale_search(W, H, alpha, all_err=True)
+    _, idx1, _ = oracle_mod.refine(W, H, alpha, idx0, sweeps=1)
+    emin, epick = oracle_mod.refine_replay(W, H, alpha, idx0, idx1)
+    np.testing.assert_array_equal(emin, epick)
+    assert np.any(idx1 != idx0)
