@@ -239,6 +239,31 @@ qat4_status qat4_scale_search_rowwise(const float *W, int64_t R, int64_t C,
                                       float *delta, int32_t *idx, float *best_err,
                                       void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* ------------------------------------------------ full-objective refinement
+ * The model card ("Quantization Configuration") writes the scale objective
+ * over the whole layer, argmin ||W X - Q_Delta(W) X||_F^2: per row of W the
+ * quadratic form e H e^T of e = w - Q_Delta(w) over all C columns, including
+ * the cross-group blocks of H that qat4_scale_search leaves out.  Starting
+ * from the given candidate indices (normally the search's), each of `sweeps`
+ * passes visits the groups of a row in order and moves each to the candidate
+ * of its own grid (Delta_k = alpha_k * fl(max|w_g| / 7)) that minimises the
+ * full objective with the other groups held; ties go to the smallest k.  The
+ * objective never increases.  Arithmetic: exact codes, exact binary64 errors,
+ * binary64 objective differences (v = H e kept per row).
+ *  W      float32 [R, C];  H float32 [C, C] (row stride ldh >= C, ldh % 4 == 0),
+ *         symmetric (as qat4_hessian writes it);  alpha float32 [K].
+ *  idx    int32 [R, C/32], in: start indices in [0, K) (others are clamped),
+ *         out: refined indices.
+ *  delta  out float32 [R, C/32]: alpha[idx] * fl(max|w_g| / 7).
+ *  obj    out float64 [R] (nullable): the final e H e^T of every row.
+ *  workspace  >= qat4_refine_workspace_bytes(R, C) bytes (2 R C binary64).
+ *  sweeps >= 0 (0 only evaluates the start).
+ *  Errors: QAT4_ERR_NULL, _SHAPE, _ALIGN, _WORKSPACE, _CUDA. */
+size_t qat4_refine_workspace_bytes(int64_t R, int64_t C);
+qat4_status qat4_refine(const float *W, int64_t R, int64_t C, const float *H, int64_t ldh, const float *alpha,
+                        int32_t K, int32_t sweeps, int32_t *idx, float *delta, double *obj, void *workspace,
+                        size_t workspace_bytes, cudaStream_t stream);
+
 /* ---------------------------------------------------------------- inference
  * The product on the W4A16 export (model card "Opt.Gear-1B-qat-int4-per-
  * channel-unquantized", section "Quantization Configuration": INT4 weights,

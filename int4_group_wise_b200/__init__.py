@@ -49,6 +49,8 @@ EXPORTS = {
     "qat4_scale_search_rowwise": (ct.c_int, [_P, _I64, _I64, _P, _I64, _P, _I32, _P, _P, _P, _P, _Z, _P]),
     "qat4_w4a16_gemv": (ct.c_int, [_P, _I64, _P, _P, _I64, _I64, _I64, _P, _P]),
     "qat4_fq_gemm": (ct.c_int, [_P, _I64, _P, _P, _I64, _I64, _P, _P]),
+    "qat4_refine_workspace_bytes": (ct.c_size_t, [_I64, _I64]),
+    "qat4_refine": (ct.c_int, [_P, _I64, _I64, _P, _I64, _P, ct.c_int32, ct.c_int32, _P, _P, _P, _P, _Z, _P]),
     "qat4_sync_check": (ct.c_int, [_P]),
     "qat4_selftest_bounded_wait": (ct.c_int, [_I64, _P]),
 }
@@ -384,6 +386,28 @@ def fq_gemm(X, W, delta, Y=None, stream=None):
     _check(L.qat4_fq_gemm(_dev(X, "X"), T, _dev(W, "W"), _dev(delta, "delta"), R, C, _dev(Y, "Y"),
                           _stream(stream)), "qat4_fq_gemm")
     return Y
+
+
+def refine(W, H, alpha, idx, sweeps=1, delta=None, obj=None, workspace=None, stream=None):
+    """Full-objective coordinate descent over the groups of each row, starting from idx (int32
+    [R, C/32], refined in place); returns (delta float32 [R, C/32], idx, obj float64 [R])."""
+    import torch
+    L = lib()
+    _dev(W, "W", torch.float32)
+    R, C = W.shape
+    _dev(H, "H", torch.float32)
+    _dev(alpha, "alpha", torch.float32)
+    _dev(idx, "idx", torch.int32, (R, C // 32))
+    delta = _out(delta, "delta", (R, C // 32), torch.float32, W)
+    obj = _out(obj, "obj", (R,), torch.float64, W)
+    need = L.qat4_refine_workspace_bytes(R, C)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=W.device)
+    _check(L.qat4_refine(_dev(W, "W"), R, C, _dev(H, "H"), H.shape[1], _dev(alpha, "alpha"), alpha.numel(),
+                         int(sweeps), _dev(idx, "idx"), _dev(delta, "delta"), _dev(obj, "obj"),
+                         _dev(workspace, "workspace", torch.uint8), workspace.numel(), _stream(stream)),
+           "qat4_refine")
+    return delta, idx, obj
 
 
 def sync_check(stream=None):

@@ -21,6 +21,7 @@
 #include "rowwise_search.cuh"
 #include "w4a16_gemv.cuh"
 #include "fq_gemm.cuh"
+#include "refine.cuh"
 
 namespace {
 
@@ -556,6 +557,43 @@ qat4_status qat4_fq_gemm(const uint16_t* X, int64_t T, const float* W, const flo
     p.limit_ns = 4000000000ull + 10000ull * static_cast<uint64_t>(p.ksteps);
     const unsigned grid = static_cast<unsigned>(2 * tiles_m * tiles_r);
     qat4::fq_gemm_kernel<<<grid, qat4::kFqThreads, qat4::kFqSmemBytes, stream>>>(tx, tw, p);
+    return launch_status();
+}
+
+// ------------------------------------------------------ full-objective refinement
+size_t qat4_refine_workspace_bytes(int64_t R, int64_t C) {
+    if (!valid_rc(R, C)) return 0;
+    return 2 * static_cast<size_t>(R) * static_cast<size_t>(C) * sizeof(double);
+}
+
+qat4_status qat4_refine(const float* W, int64_t R, int64_t C, const float* H, int64_t ldh, const float* alpha,
+                        int32_t K, int32_t sweeps, int32_t* idx, float* delta, double* obj, void* workspace,
+                        size_t workspace_bytes, cudaStream_t stream) {
+    if (!W || !H || !alpha || !idx || !delta) return QAT4_ERR_NULL;
+    if (!valid_rc(R, C) || K < 1 || sweeps < 0 || ldh < C || R > 65535 * int64_t(qat4::kRfTile))
+        return QAT4_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(H) || !aligned16(alpha) || !aligned16(idx) || !aligned16(delta) ||
+        (obj && !aligned16(obj)) || (ldh % 4) != 0 || (workspace && !aligned16(workspace)))
+        return QAT4_ERR_ALIGN;
+    const size_t need = qat4_refine_workspace_bytes(R, C);
+    if (!workspace || workspace_bytes < need) return QAT4_ERR_WORKSPACE;
+    int dev = 0;
+    DeviceInfo* info = nullptr;
+    if (!device_info(&dev, &info)) return QAT4_ERR_CUDA;
+    double* E = static_cast<double*>(workspace);
+    double* V = E + R * C;
+    const int64_t ngroups = R * (C / 32);
+    const int64_t err_blocks = (ngroups + 7) / 8;
+    const unsigned eb = static_cast<unsigned>(err_blocks < int64_t(info->sms) * 16 ? err_blocks : int64_t(info->sms) * 16);
+    qat4::refine_err_kernel<<<eb, 256, 0, stream>>>(W, ngroups, alpha, K, idx, E);
+    if (cudaGetLastError() != cudaSuccess) return QAT4_ERR_CUDA;
+    const dim3 vgrid(static_cast<unsigned>((C + qat4::kRfTile - 1) / qat4::kRfTile),
+                     static_cast<unsigned>((R + qat4::kRfTile - 1) / qat4::kRfTile));
+    qat4::refine_v_kernel<<<vgrid, 256, 0, stream>>>(E, static_cast<int>(R), static_cast<int>(C), H, ldh, V);
+    if (cudaGetLastError() != cudaSuccess) return QAT4_ERR_CUDA;
+    const unsigned sgrid = static_cast<unsigned>((R + qat4::kRfWarps - 1) / qat4::kRfWarps);
+    qat4::refine_sweep_kernel<<<sgrid, 32 * qat4::kRfWarps, 0, stream>>>(
+        W, static_cast<int>(R), static_cast<int>(C), H, ldh, alpha, K, sweeps, idx, delta, obj, V);
     return launch_status();
 }
 

@@ -117,3 +117,14 @@ def test_hessian_partial_validation():
     assert L.qat4_hessian_partial(A, 64, 64, 63, A, None, 0, None) == 2      # n_total < n
     assert L.qat4_hessian_partial(A, 64, 40, 64, A, None, 0, None) == 2
     assert L.qat4_hessian_partial(MIS, 64, 64, 128, A, None, 0, None) == 3
+
+
+def test_refine_validation():
+    L = q4.lib()
+    assert L.qat4_refine(None, 4, 64, A, 64, A, 5, 1, A, A, None, A, 1 << 20, None) == 1
+    assert L.qat4_refine(A, 4, 64, A, 64, A, 0, 1, A, A, None, A, 1 << 20, None) == 2      # K = 0
+    assert L.qat4_refine(A, 4, 64, A, 64, A, 5, -1, A, A, None, A, 1 << 20, None) == 2     # sweeps < 0
+    assert L.qat4_refine(A, 4, 64, A, 32, A, 5, 1, A, A, None, A, 1 << 20, None) == 2      # ldh < C
+    assert L.qat4_refine(A, 4, 64, A, 66, A, 5, 1, A, A, None, A, 1 << 20, None) == 3      # ldh % 4
+    assert L.qat4_refine(A, 4, 64, A, 64, A, 5, 1, A, A, None, A, 16, None) == 5           # workspace
+    assert L.qat4_refine_workspace_bytes(4, 64) == 2 * 4 * 64 * 8
