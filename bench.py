@@ -816,6 +816,79 @@ def run_hessian_split(args):
         dist.destroy_process_group()
 
 
+def run_refine(args):
+    """The full-objective refinement (one coordinate-descent sweep over the groups of every row)
+    on the 1B-class up-projection, starting from the GPU search's indices; each launch timed with
+    CUDA events after an L2 flush.  Work model in binary64 FMAs: V = E H (R C^2), every
+    candidate of every group (R G K (528 + 32)) and the v updates of the groups that move
+    (moves x 32 C)."""
+    import torch
+
+    import int4_group_wise_b200 as q4
+    from int4_group_wise_b200 import inputs
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peaks, peak_kind = load_peaks()
+    wl = inputs.workload(1)
+    m = wl.matrices[0]
+    W = torch.from_numpy(wl.weight(m)).to(dev)
+    R, C = W.shape
+    X = torch.from_numpy(wl.activations(m.x_name).view(np.int16)).to(dev).view(torch.bfloat16)
+    H = q4.hessian(X)
+    del X
+    alpha = torch.from_numpy(wl.alpha()).to(dev)
+    K = alpha.numel()
+    _, idx0, _ = q4.scale_search(W, H, alpha)
+    idx = idx0.clone()
+    delta = torch.empty((R, C // 32), dtype=torch.float32, device=dev)
+    obj = torch.empty((R,), dtype=torch.float64, device=dev)
+    ws = torch.empty(q4.lib().qat4_refine_workspace_bytes(R, C), dtype=torch.uint8, device=dev)
+    q4.refine(W, H, alpha, idx, 0, delta, obj, ws)
+    obj0 = obj.clone()
+    flush_buf = torch.ones(128 << 20, dtype=torch.float32, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def one():
+        idx.copy_(idx0)
+        q4.refine(W, H, alpha, idx, 1, delta, obj, ws)
+
+    for _ in range(args.warmup):
+        one()
+    q4.sync_check()
+    ts = []
+    with ClockSampler(0) as clk:
+        for _ in range(args.steps):
+            idx.copy_(idx0)
+            torch.sum(flush_buf, dim=0, out=sink)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            q4.refine(W, H, alpha, idx, 1, delta, obj, ws)
+            b.record(stream)
+            ts.append((a, b))
+        torch.cuda.synchronize()
+    q4.sync_check()
+    ms = statistics.median(a.elapsed_time(b) for a, b in ts)
+    G = C // 32
+    moves = int((idx != idx0).sum().item())
+    dfma = float(R) * C * C + float(R) * G * K * 560 + float(moves) * 32 * C
+    fp64_peak = 148 * 64 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6
+    gain = (1.0 - obj / obj0)
+    print(json.dumps({
+        "metric": "full-objective refinement, one sweep: groups/s", "value": R * G / ms * 1e3, "unit": "groups/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "variant": "refine", "data": "synthetic", "dtype": "f64 (exact f32 codes)",
+        "config": {"workload": f"1B-class up-projection W fp32 {R}x{C}, H of 262144 calibration rows, K={K}",
+                   "l2": "flushed (512 MB read sweep) before every launch"},
+        "roofline": {"bound": "fp64", "achieved": dfma / (ms * 1e-3) / 1e12, "peak": fp64_peak / 1e12,
+                     "unit": "T FMA/s", "frac": dfma / (ms * 1e-3) / fp64_peak,
+                     "peak_kind": "148 SM x 64 FP64 FMA/clock at max SM clock"},
+        "fp64_fma_per_launch": dfma, "groups_moved": moves, "groups": R * G,
+        "objective_gain_median": float(gain.median().item()), "objective_gain_max": float(gain.max().item()),
+        "gpu_launches": 3 * args.steps, "clocks": clk.summary()}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -824,12 +897,14 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--variant", choices=["group32", "per-channel", "w4a16-decode", "fq-gemm", "hessian-split"],
+    ap.add_argument("--variant", choices=["group32", "per-channel", "w4a16-decode", "fq-gemm", "hessian-split",
+                                          "refine"],
                     default="group32",
                     help="per-channel: time the one-scale-per-row LSQ step and export instead; "
                          "w4a16-decode: time the inference GEMV on the packed 8B-class stack; "
                          "fq-gemm: time the fused fake-quant forward GEMM; "
-                         "hessian-split: the calibration Hessian with its rows split over the ranks")
+                         "hessian-split: the calibration Hessian with its rows split over the ranks; "
+                         "refine: one sweep of the full-objective refinement")
     ap.add_argument("--tokens", type=int, default=8192, help="fq-gemm: tokens of the micro-batch")
     ap.add_argument("--layers", type=int, default=None,
                     help="w4a16-decode: number of layers of the 8B-class stack (default: all 32)")
@@ -846,6 +921,8 @@ def main():
         run_fq_gemm(args)
     elif args.variant == "hessian-split":
         run_hessian_split(args)
+    elif args.variant == "refine":
+        run_refine(args)
     else:
         run_ours(args)
 
