@@ -269,7 +269,7 @@ qat4_status qat4_refine(const float *W, int64_t R, int64_t C, const float *H, in
  * channel-unquantized", section "Quantization Configuration": INT4 weights,
  * 16-bit activations), for decode-sized batches:
  *     y[m, r] = sum_c x[m, c] * (scale[r, c / group] * code[r, c])
- *  x       bf16 bit patterns [M, C] (M tokens, 1 <= M <= 65535; processed up to four
+ *  x       bf16 bit patterns [M, C] (M tokens, 1 <= M <= 65535; processed up to eight
  *          tokens per pass -- fewer when x of a wide row does not fit shared memory -- so
  *          the codes are read once per pass).
  *  packed  uint8 [R, C/2], the layout of qat4_pack_w4a16 (element 2j in the low nibble of
@@ -278,9 +278,10 @@ qat4_status qat4_refine(const float *W, int64_t R, int64_t C, const float *H, in
  *          qat4_pack_w4a16, group = C for qat4_pack_w4a16_rowwise (any multiple of 32 that
  *          divides C is accepted).
  *  y       out float32 [M, R]; zeroed on the stream first, then written.  Products are
- *          exact, sums float32 in an order fixed by (R, C, M) and the SM count.
- *  C must be a multiple of 32 and small enough that one token's x (bf16) and two 32 KB
- *  stages fit the opt-in shared memory of a block (C <= 83296 on B200); else _SHAPE.
+ *          exact (bf16 codes times bf16 x on the tensor cores), sums float32 in an order
+ *          fixed by (R, C, M) and the SM count.
+ *  C must be a multiple of 32 and small enough that one token's x (bf16) and three 16 KB
+ *  stages fit the opt-in shared memory of a block (C <= 88064 on B200); else _SHAPE.
  *  Errors: QAT4_ERR_NULL, _SHAPE, _ALIGN, _CUDA. */
 qat4_status qat4_w4a16_gemv(const uint16_t *x, int64_t M, const uint8_t *packed, const uint16_t *scales,
                             int64_t R, int64_t C, int64_t group, float *y, cudaStream_t stream);

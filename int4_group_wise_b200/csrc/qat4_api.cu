@@ -429,72 +429,63 @@ qat4_status qat4_w4a16_gemv(const uint16_t* x, int64_t M, const uint8_t* packed,
             int optin = 0;
             if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
                 return QAT4_ERR_CUDA;
-            if (cudaFuncSetAttribute(qat4::w4a16_gemv_kernel<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) ||
-                cudaFuncSetAttribute(qat4::w4a16_gemv_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) ||
-                cudaFuncSetAttribute(qat4::w4a16_gemv_kernel<1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) ||
-                cudaFuncSetAttribute(qat4::w4a16_gemv_kernel<2, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) ||
-                cudaFuncSetAttribute(qat4::w4a16_gemv_kernel<3, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin) ||
-                cudaFuncSetAttribute(qat4::w4a16_gemv_kernel<4, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, optin))
+            if (cudaFuncSetAttribute(qat4::w4a16_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, optin))
                 return QAT4_ERR_CUDA;
             info->smem_optin = optin;
         }
     }
     const size_t optin = static_cast<size_t>(info->smem_optin);
-    // tokens per pass: up to 4, fewer when x (bf16) of a wider C leaves under two ring slots;
-    // a pass keeps x in float32 when that still leaves two slots
-    int mt_max = 4;
-    while (mt_max > 0 && qat4::gemv_smem_bytes(mt_max, false, static_cast<int>(C), 2) > optin) --mt_max;
+    const int c = static_cast<int>(C);
+    // tokens per pass: up to 8, fewer when x of a wide row leaves under three ring slots
+    int mt_max = qat4::kGmMaxTokens;
+    while (mt_max > 0 && qat4::gemv_smem_bytes(mt_max, c, 3) > optin) --mt_max;
     if (mt_max == 0) return QAT4_ERR_SHAPE;
 
     EncodeTiledFn encode = encode_tiled();
     if (!encode) return QAT4_ERR_CUDA;
+    CUtensorMap tmap;   // codes as uint32 words [R, C/8]; one box = 16 rows x 128 bytes, 128-byte swizzle
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(C / 8), static_cast<cuuint64_t>(R)};
+        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(C / 2)};
+        const cuuint32_t box[2] = {32, static_cast<cuuint32_t>(qat4::kGmRows)};
+        const cuuint32_t estr[2] = {1, 1};
+        if (encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t*>(packed), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return QAT4_ERR_CUDA;
+    }
     if (cudaMemsetAsync(y, 0, static_cast<size_t>(M) * static_cast<size_t>(R) * sizeof(float), stream) != cudaSuccess)
         return QAT4_ERR_CUDA;
     qat4::GemvParams p;
     p.scales = scales;
     p.R = static_cast<int>(R);
-    p.C = static_cast<int>(C);
+    p.C = c;
     p.group = static_cast<int>(group);
     p.G = static_cast<int>(C / group);
-    p.nchunks = static_cast<int>((C + qat4::kGvChunkCols - 1) / qat4::kGvChunkCols);
-    const uint32_t dmask[5] = {0xFu, 0xF0u, 0xF00u, 0xF000u, 0xF0000u};
-    // bit pattern of 2^(23 - 4k), plus the top bit of nibble k
-    const uint32_t dbits[5] = {0x4B000008u, 0x49000080u, 0x47000800u, 0x45008000u, 0x43080000u};
-    for (int k = 0; k < 5; ++k) {
-        p.dmask[k] = dmask[k];
-        p.dbits[k] = dbits[k];
-    }
+    p.nblocks = static_cast<int>((R + qat4::kGmRows - 1) / qat4::kGmRows);
+    p.nchunks = static_cast<int>((C + qat4::kGmChunkCols - 1) / qat4::kGmChunkCols);
+    p.xstride = qat4::gemv_xstride(c);
+    p.dmask = 0x000F000Fu;        // nibbles at bits 0..3 and 16..19
+    p.dbits = 0x43084308u;        // bf16 exponent of 128 in both halves, plus the nibbles' top bit
     for (int64_t m0 = 0; m0 < M; m0 += mt_max) {
         const int mt = static_cast<int>(M - m0 < mt_max ? M - m0 : mt_max);
-        const int rb = qat4::gemv_row_block(mt);
-        CUtensorMap tmap;   // codes as uint32 words [R, C/8], one box = rb rows x 512 bytes
-        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(C / 8), static_cast<cuuint64_t>(R)};
-        const cuuint64_t strides[1] = {static_cast<cuuint64_t>(C / 2)};
-        const cuuint32_t box[2] = {qat4::kGvRowBytes / 4, static_cast<cuuint32_t>(rb)};
-        const cuuint32_t estr[2] = {1, 1};
-        if (encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint8_t*>(packed), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return QAT4_ERR_CUDA;
-        p.nblocks = static_cast<int>((R + rb - 1) / rb);
-        const int grid = p.nblocks < info->sms ? p.nblocks : info->sms;   // ranges >= one row block
+        // two CTAs per SM when two 5-stage rings fit, else one with as many stages as fit
+        int per_sm = 2, stages = 5;
+        if (2 * (qat4::gemv_smem_bytes(mt, c, stages) + 1024) > 228u * 1024u) {
+            per_sm = 1;
+            stages = qat4::kGmMaxStages;
+            while (stages > 3 && qat4::gemv_smem_bytes(mt, c, stages) > optin) --stages;
+        }
+        const int64_t want = static_cast<int64_t>(info->sms) * per_sm;
+        const int grid = static_cast<int>(p.nblocks < want ? p.nblocks : want);   // ranges >= one row block
         const int64_t per_cta = (static_cast<int64_t>(p.nblocks) * p.nchunks + grid - 1) / grid;
         // generous bound: 4 s plus 20 us per stage of a CTA (a stage streams in well under 1 us)
         p.limit_ns = 4000000000ull + 20000ull * static_cast<uint64_t>(per_cta);
-        const bool xf32 = mt <= 2 && qat4::gemv_smem_bytes(mt, true, p.C, 2) <= optin;
-        int stages = qat4::kGvMaxStages;
-        while (stages > 2 && qat4::gemv_smem_bytes(mt, xf32, p.C, stages) > optin) --stages;
         p.stages = stages;
+        p.MT = mt;
         p.x = x + m0 * C;
         p.y = y + m0 * R;
-        const size_t smem = qat4::gemv_smem_bytes(mt, xf32, p.C, stages);
-        const unsigned th = qat4::kGvThreads;
-        if (mt == 1 && xf32) qat4::w4a16_gemv_kernel<1, true><<<grid, th, smem, stream>>>(tmap, p);
-        else if (mt == 2 && xf32) qat4::w4a16_gemv_kernel<2, true><<<grid, th, smem, stream>>>(tmap, p);
-        else if (mt == 1) qat4::w4a16_gemv_kernel<1, false><<<grid, th, smem, stream>>>(tmap, p);
-        else if (mt == 2) qat4::w4a16_gemv_kernel<2, false><<<grid, th, smem, stream>>>(tmap, p);
-        else if (mt == 3) qat4::w4a16_gemv_kernel<3, false><<<grid, th, smem, stream>>>(tmap, p);
-        else qat4::w4a16_gemv_kernel<4, false><<<grid, th, smem, stream>>>(tmap, p);
+        qat4::w4a16_gemv_kernel<<<grid, qat4::kGmThreads, qat4::gemv_smem_bytes(mt, c, stages), stream>>>(tmap, p);
         if (cudaGetLastError() != cudaSuccess) return QAT4_ERR_CUDA;
     }
     return QAT4_OK;

@@ -1,148 +1,183 @@
 // w4a16_gemv.cuh -- the inference product on the W4A16 export (model card
 // "Opt.Gear-1B-qat-int4-per-channel-unquantized", section "Quantization
 // Configuration": INT4 weights with 16-bit activations; "QAT Highlights": the
-// learned grid survives export).  For a decode batch of MT <= 4 tokens:
+// learned grid survives export).  For a decode batch of MT <= 8 tokens:
 //     y[m, r] = sum_c x[m, c] * (scale[r, c / group] * code[r, c])
 // with x in bf16, the codes and binary16 scales of the packed export (element
-// 2j in the low nibble of byte j), and float32 accumulation.  The kernel reads
-// the 0.5 B of codes and 2/group B of scale of every weight once: HBM-bound.
+// 2j in the low nibble of byte j), products exact and float32 sums.  The
+// kernel reads the 0.5 B of codes and 2/group B of scale of every weight once:
+// it is HBM-bound, so its inner products go to the tensor cores only to take
+// the multiply-adds off the issue slots that the decoding needs.
 //
-// Data movement.  A persistent grid (one CTA per SM) walks the list of
-// "stages" (row block) x (column chunk of 1024 columns), cut into equal
-// contiguous ranges, one per CTA.  A producer warp streams each stage's codes
-// (512 B per row) into a ring of shared-memory slots with 2-D bulk-tensor
-// copies (no multicast); sixteen consumer warps take RPW rows each (4, or 2
-// above two tokens), so a row block is 64 or 32 rows.
-// The CTA's x (all MT tokens, all C columns) is staged in shared memory once:
-// converted to float32 when it fits (MT <= 2), else kept as bf16; the 16-byte
-// slots of every 32-column quad are XOR-swizzled by the quad index, so that
-// the 32 lanes of a warp (lane l on quad l of the chunk) read x without bank
-// conflicts.  Each x load serves the warp's RPW rows.
+// Tensor cores.  mma.sync m16n8k16 (bf16 x bf16 -> f32): A = 16 rows of W by
+// 16 columns of codes (exact small integers in bf16), B = 16 columns of x by 8
+// tokens (tokens past MT are zero), D in registers.  Two MMAs cover one
+// 32-column group; their D is scaled by the group's scale into a float32
+// accumulator.  The 16 columns of one MMA are a permutation of the group's
+// columns, the same for A and B: lane (g, t) takes word t of the group (its 8
+// nibbles, columns 8t..8t+7) for rows g and g+8, and the MMA's column pairs
+// (2t, 2t+1) and (2t+8, 2t+9) are nibbles (0, 4) and (1, 5) in the first MMA,
+// (2, 6) and (3, 7) in the second.  x is staged with every 8-column word in
+// the order (0, 4, 1, 5, 2, 6, 3, 7), so one 16-byte load gives a lane both
+// MMAs' B registers.
 //
-// Decoding without int -> float conversions.  Nibble k of a 32-bit word,
-// masked in place with its top bit flipped (code + 8) and placed into the bit
-// pattern of 2^(23 - 4k), is the float 2^(23-4k) + code + 8 exactly (the
-// mantissa unit at that exponent is 2^-4k); subtracting 2^(23-4k) + 8 leaves
-// the code.  Mask, flip and exponent are one three-input logic op.  Nibbles 0..4 use the word itself, nibbles
-// 5..7 the word shifted right by 16 (back at bits 4..15).  Products x * code
-// are exact; they are summed with packed FP32x2 FMAs over the 32 weights of a
-// quad, then scaled by the group's scale.
+// Decoding.  One three-input logic op turns the nibbles at bits 0..3 and
+// 16..19 of a word (shifted right by 0, 4, 8 or 12) into two bf16 values
+// 128 + (code + 8) -- the nibble with its top bit flipped, under the exponent
+// of 128 -- and one packed bf16 subtraction of 136 leaves the two codes,
+// exactly.
 //
-// Partial rows.  A row block cut between two CTAs gets one partial sum from
-// each; both are added atomically into y, which the host zeroes first.  The
-// ranges are at least one row block long, so no row has more than two
-// contributions, and fl(0 + a + b) does not depend on their order: the result
-// is deterministic.
+// Data movement.  A persistent grid walks the list of stages (block of 16 rows)
+// x (chunk of 2048 columns), cut into equal contiguous ranges of at least one
+// row block, one per CTA.  A producer warp streams each stage's codes as eight
+// 16-row x 128-byte boxes (2-D bulk-tensor copies, 128-byte swizzle, no
+// multicast) into a ring of shared-memory slots; eight consumer warps take 8
+// groups each, so a lane reads its 4-byte words of 8 rows from 8 different
+// bank groups.  At the end of a row block the warps' partial tiles are summed
+// in shared memory in a fixed order.  A row block cut between two CTAs gets one
+// partial sum from each, added atomically into y (zeroed by the host): with at
+// most two contributions, fl(0 + a + b) does not depend on their order.
 #pragma once
 
 #include <cuda.h>
+#include <cuda_bf16.h>
 
 #include "device_common.cuh"
 
 namespace qat4 {
 
-constexpr int kGvConsumerWarps = 16;
-constexpr int kGvThreads = 32 * (kGvConsumerWarps + 1);            // + one producer warp
-constexpr int kGvChunkCols = 1024;                                  // columns per stage
-constexpr int kGvRowBytes = kGvChunkCols / 2;                       // 512 B of codes per row and stage
-constexpr int kGvMaxStages = 12;
-constexpr uint64_t kGvDrainLimitNs = 1000000000ull;
-
-// Rows per consumer warp (the reuse of each x load) for MT tokens: 4, or 2 when MT > 2 so that
-// the accumulators of 16 warps fit the register file.
-__host__ __device__ constexpr int gemv_rows_per_warp(int MT) { return MT <= 2 ? 4 : 2; }
-__host__ __device__ constexpr int gemv_row_block(int MT) { return kGvConsumerWarps * gemv_rows_per_warp(MT); }
-__host__ __device__ constexpr int gemv_stage_bytes(int MT) { return gemv_row_block(MT) * kGvRowBytes; }
-
+constexpr int kGmWarps = 8;                                 // consumer warps
+constexpr int kGmThreads = 32 * (kGmWarps + 1);             // + one producer warp
+constexpr int kGmRows = 16;                                 // rows per block (one MMA tile)
+constexpr int kGmChunkCols = 2048;                          // columns per stage
+constexpr int kGmBoxBytes = kGmRows * 128;                  // 16 rows x 256 columns of codes
+constexpr int kGmStageBytes = 8 * kGmBoxBytes;              // 16 KB
+constexpr int kGmMaxStages = 12;
+constexpr int kGmQuads = kGmChunkCols / 32 / kGmWarps;      // groups per warp and stage (8)
+constexpr int kGmMaxTokens = 8;
+constexpr uint64_t kGmDrainLimitNs = 1000000000ull;
 
 struct GemvParams {
     const uint16_t* x;       // bf16 bits [MT, C], row stride C
     const uint16_t* scales;  // binary16 bits [R, C / group]
     float* y;                // [MT, R], zeroed by the host
     int R, C, group, G;      // G = C / group
-    int nblocks, nchunks;    // row blocks of gemv_row_block(MT) rows, column chunks of 1024
+    int MT;                  // tokens of this pass, 1..8
+    int nblocks, nchunks;    // blocks of 16 rows, chunks of 2048 columns
     int stages;              // ring slots
+    int xstride;             // bytes per staged token row
     uint64_t limit_ns;
-    // nibble masks and exponent-and-flip patterns of the decode, filled by the host so that
-    // they stay register operands of one three-input logic op each
-    uint32_t dmask[5], dbits[5];
+    // mask and exponent-and-flip pattern of the decode, filled by the host so that they stay
+    // register operands of one three-input logic op
+    uint32_t dmask, dbits;
 };
 
-// Bytes of x in shared memory per column: float32 (converted once while staging) or bf16.
-__host__ __device__ constexpr int gemv_x_bytes(bool xf32) { return xf32 ? 4 : 2; }
-
-// Shared-memory bytes of the kernel for MT tokens, C columns and `stages` ring slots.
-__host__ __device__ constexpr size_t gemv_smem_bytes(int MT, bool xf32, int C, int stages) {
-    return static_cast<size_t>(stages) * gemv_stage_bytes(MT) + static_cast<size_t>(MT) * C * gemv_x_bytes(xf32) +
-           static_cast<size_t>(2 * kGvMaxStages) * 8 + 128;
+// Bytes per staged token row of x: the columns rounded up to whole chunks, 8 bf16 per 16 bytes,
+// plus 64 bytes so that consecutive tokens start in different bank groups.
+__host__ __device__ constexpr int gemv_xstride(int C) {
+    return ((C + kGmChunkCols - 1) / kGmChunkCols) * kGmChunkCols * 2 + 64;
 }
 
-// Byte offset, in one token's row of x, of 16-byte slot j of the 32-column quad q: 8 slots of
-// 4 floats (float32 x) or 4 slots of 8 bf16, XOR-swizzled by the quad index so that 32 lanes
-// on 32 consecutive quads hit distinct banks.
-__host__ __device__ constexpr uint32_t gv_xslot_f32(uint32_t q, uint32_t j) { return q * 128u + 16u * (j ^ (q & 7u)); }
-__host__ __device__ constexpr uint32_t gv_xslot_bf16(uint32_t q, uint32_t j) {
-    return q * 64u + 16u * (j ^ ((q >> 1) & 3u));
+// Shared-memory bytes of the kernel for MT tokens, C columns and `stages` ring slots.
+__host__ __device__ constexpr size_t gemv_smem_bytes(int MT, int C, int stages) {
+    return 1024 + static_cast<size_t>(stages) * kGmStageBytes + static_cast<size_t>(MT) * gemv_xstride(C) +
+           static_cast<size_t>(kGmWarps) * 32 * 4 * 4 + static_cast<size_t>(2 * kGmMaxStages) * 8 + 16;
 }
 
 // (a & m) ^ c as one three-input logic op.
-__device__ __forceinline__ uint32_t gv_and_xor(uint32_t a, uint32_t m, uint32_t c) {
+__device__ __forceinline__ uint32_t gm_and_xor(uint32_t a, uint32_t m, uint32_t c) {
     uint32_t d;
     asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(m), "r"(c));
     return d;
 }
 
-// The 8 codes of one word as 4 float pairs (nibbles 0,1 | 2,3 | 4,5 | 6,7).  Nibbles 0..4 are
-// taken from the word, nibbles 5..7 from the word shifted right by 16 (back at bits 4..15).
-struct GvDec { uint32_t m[5], c[5]; };
-__device__ __forceinline__ void gv_decode(uint32_t w, const GvDec& d, float2 (&v)[4]) {
-    const uint32_t hi = w >> 16;
-    const float2 f01 = make_float2(__uint_as_float(gv_and_xor(w, d.m[0], d.c[0])),
-                                   __uint_as_float(gv_and_xor(w, d.m[1], d.c[1])));
-    const float2 f23 = make_float2(__uint_as_float(gv_and_xor(w, d.m[2], d.c[2])),
-                                   __uint_as_float(gv_and_xor(w, d.m[3], d.c[3])));
-    const float2 f45 = make_float2(__uint_as_float(gv_and_xor(w, d.m[4], d.c[4])),
-                                   __uint_as_float(gv_and_xor(hi, d.m[1], d.c[1])));
-    const float2 f67 = make_float2(__uint_as_float(gv_and_xor(hi, d.m[2], d.c[2])),
-                                   __uint_as_float(gv_and_xor(hi, d.m[3], d.c[3])));
-    // 2^23 + 8, 2^19 + 8, 2^15 + 8, 2^11 + 8, 2^7 + 8
-    v[0] = __fadd2_rn(f01, make_float2(-8388616.0f, -524296.0f));
-    v[1] = __fadd2_rn(f23, make_float2(-32776.0f, -2056.0f));
-    v[2] = __fadd2_rn(f45, make_float2(-136.0f, -524296.0f));
-    v[3] = __fadd2_rn(f67, make_float2(-32776.0f, -2056.0f));
+// Codes of the nibbles at bits 0..3 and 16..19 of v, as a bf16 pair (low half first).
+__device__ __forceinline__ uint32_t gm_pair(uint32_t v, uint32_t m, uint32_t c) {
+    __nv_bfloat162 h;
+    *reinterpret_cast<uint32_t*>(&h) = gm_and_xor(v, m, c);                 // 128 + (code + 8)
+    const __nv_bfloat162 r = __hsub2(h, __floats2bfloat162_rn(136.0f, 136.0f));
+    return *reinterpret_cast<const uint32_t*>(&r);
 }
 
-// Scales of the warp's RPW rows for the quad of `lane` in stage (b, ch); 0 past the matrix.
-template <int RPW>
-__device__ __forceinline__ void gv_scales(const uint16_t* __restrict__ scales, int R, int G, int C, int group,
-                                          int b, int ch, int row0, int lane, float (&s)[RPW]) {
-    const int q = ch * (kGvChunkCols / 32) + lane;
-    const bool in = q < (C >> 5);
-    const int g = group == 32 ? q : (q * 32) / group;
+__device__ __forceinline__ void gm_mma(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t gm_lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint4 gm_lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+
+// Scales of rows (g, g+8) of block b for the kGmQuads groups of warp `warp` in chunk ch, in the
+// order (row g, row g+8) per group; 0 past the matrix.  The group-32 export reads the 8 scales of
+// a row with one 16-byte load (no division), the per-row export one scale per row.
+struct GmScaleCtx {
+    const uint16_t* scales;
+    int R, C, G, group, warp, g;
+    bool fast32;             // group 32 and G % 8 == 0
+};
+__device__ __forceinline__ float gm_half(uint32_t v, int hi) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(hi ? v >> 16 : v & 0xFFFFu)));
+}
+__device__ __forceinline__ void gm_scales(const GmScaleCtx& x, int b, int ch, float (&s)[2 * kGmQuads]) {
+    const int ra = b * kGmRows + x.g, rb = ra + 8;
+    const int q0 = ch * (kGmChunkCols / 32) + kGmQuads * x.warp;   // this warp's first group of 32 columns
+    if (x.fast32 && q0 + kGmQuads <= x.G) {
+        uint4 va = make_uint4(0u, 0u, 0u, 0u), vb = make_uint4(0u, 0u, 0u, 0u);
+        if (ra < x.R) va = __ldg(reinterpret_cast<const uint4*>(x.scales + static_cast<int64_t>(ra) * x.G + q0));
+        if (rb < x.R) vb = __ldg(reinterpret_cast<const uint4*>(x.scales + static_cast<int64_t>(rb) * x.G + q0));
+        const uint32_t a4[4] = {va.x, va.y, va.z, va.w}, b4[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
-    for (int i = 0; i < RPW; ++i) {
-        const int r = b * kGvConsumerWarps * RPW + row0 + i;
-        s[i] = (r < R && in) ? __half2float(__ushort_as_half(__ldg(scales + static_cast<int64_t>(r) * G + g)))
-                             : 0.0f;
+        for (int j = 0; j < kGmQuads; ++j) {
+            s[2 * j] = gm_half(a4[j >> 1], j & 1);
+            s[2 * j + 1] = gm_half(b4[j >> 1], j & 1);
+        }
+        return;
+    }
+    if (x.G == 1) {
+        const float sa = ra < x.R ? __half2float(__ushort_as_half(__ldg(x.scales + ra))) : 0.0f;
+        const float sb = rb < x.R ? __half2float(__ushort_as_half(__ldg(x.scales + rb))) : 0.0f;
+#pragma unroll
+        for (int j = 0; j < kGmQuads; ++j) { s[2 * j] = sa; s[2 * j + 1] = sb; }
+        return;
+    }
+#pragma unroll
+    for (int j = 0; j < kGmQuads; ++j) {
+        const int c = (q0 + j) * 32;
+        const bool in = c < x.C;
+        const int gi = in ? c / x.group : 0;
+        s[2 * j] = (in && ra < x.R)
+                       ? __half2float(__ushort_as_half(__ldg(x.scales + static_cast<int64_t>(ra) * x.G + gi))) : 0.0f;
+        s[2 * j + 1] = (in && rb < x.R)
+                           ? __half2float(__ushort_as_half(__ldg(x.scales + static_cast<int64_t>(rb) * x.G + gi))) : 0.0f;
     }
 }
 
-template <int MT, bool XF32>
-__global__ void __launch_bounds__(kGvThreads, 1)
+__global__ void __launch_bounds__(kGmThreads)
 w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tmap, const GemvParams p) {
-    constexpr int RPW = gemv_rows_per_warp(MT);
-    constexpr int RB = gemv_row_block(MT);
-    constexpr int SB = gemv_stage_bytes(MT);
-    constexpr int XB = gemv_x_bytes(XF32);
-    extern __shared__ __align__(128) uint8_t smem[];
-    const int R = p.R, C = p.C, G = p.G, group = p.group, nchunks = p.nchunks, stages = p.stages;
-    uint8_t* ring = smem;
-    uint8_t* xs = smem + static_cast<size_t>(stages) * SB;
-    uint64_t* full_bar = reinterpret_cast<uint64_t*>(xs + static_cast<size_t>(MT) * C * XB);
-    uint64_t* empty_bar = full_bar + kGvMaxStages;
-    int* abort_flag = reinterpret_cast<int*>(empty_bar + kGvMaxStages);
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;          // the swizzle needs 1 KB alignment
+    uint8_t* smem = smem_raw + pad;
+    const uint32_t ring = raw + pad;
+    const uint32_t xs = ring + p.stages * kGmStageBytes;
+    float* red = reinterpret_cast<float*>(smem + p.stages * kGmStageBytes + p.MT * p.xstride);
+    uint64_t* full_bar = reinterpret_cast<uint64_t*>(red + kGmWarps * 32 * 4);
+    uint64_t* empty_bar = full_bar + kGmMaxStages;
+    int* abort_flag = reinterpret_cast<int*>(empty_bar + kGmMaxStages);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nchunks = p.nchunks, stages = p.stages;
     // this CTA's contiguous range of stages, at least one row block long
     const int64_t total = static_cast<int64_t>(p.nblocks) * nchunks;
     const int t0 = static_cast<int>(total * blockIdx.x / gridDim.x);
@@ -152,7 +187,7 @@ w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tmap, const GemvParams p) 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], kGvConsumerWarps);
+            mbar_init(&empty_bar[s], kGmWarps);
         }
         *abort_flag = 0;
         fence_mbar_init();
@@ -160,10 +195,9 @@ w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tmap, const GemvParams p) 
     __syncthreads();
     volatile int* abort = abort_flag;
 
-    if (warp == kGvConsumerWarps) {
+    if (warp == kGmWarps) {
         // ---------------------------------------------------------- producer
-        // lane 0 streams the codes; the lanes also pull into L2 the scales of the stage's rows,
-        // a ring's length before the consumers read them
+        // lane 0 streams the codes; lanes 0..15 also pull into L2 the scales of the stage's rows
         if (lane == 0) prefetch_tmap(&tmap);
         int issued = 0, s = 0, b = b0, ch = ch0;
         uint32_t ph = 0;
@@ -171,21 +205,20 @@ w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tmap, const GemvParams p) 
             int ok = 1;
             if (lane == 0) ok = mbar_wait(&empty_bar[s], ph ^ 1u, abort, p.limit_ns) ? 1 : 0;
             if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            const int g0 = ch * kGvChunkCols / group;
-            const int g1 = min(G, (ch * kGvChunkCols + kGvChunkCols - 1) / group + 1);
-#pragma unroll
-            for (int k = 0; k < RB / 32; ++k) {
-                const int r = b * RB + 32 * k + lane;
-                if (r < R) {
-                    const uint16_t* a = p.scales + static_cast<int64_t>(r) * G;
-                    asm volatile("prefetch.global.L2 [%0];" :: "l"(a + g0));
-                    asm volatile("prefetch.global.L2 [%0];" :: "l"(a + g1 - 1));
-                }
+            const int r = b * kGmRows + lane;
+            if (lane < kGmRows && r < p.R) {
+                const int g0 = ch * kGmChunkCols / p.group;
+                const int g1 = min(p.G, (ch * kGmChunkCols + kGmChunkCols - 1) / p.group + 1);
+                const uint16_t* a = p.scales + static_cast<int64_t>(r) * p.G;
+                asm volatile("prefetch.global.L2 [%0];" :: "l"(a + g0));
+                asm volatile("prefetch.global.L2 [%0];" :: "l"(a + g1 - 1));
             }
             if (lane == 0) {
-                mbar_arrive_expect_tx(&full_bar[s], SB);
-                // x = ch * 128 words: a multiple of 512 bytes
-                tma_load_2d(ring + static_cast<size_t>(s) * SB, &tmap, &full_bar[s], ch * (kGvRowBytes / 4), b * RB);
+                mbar_arrive_expect_tx(&full_bar[s], kGmStageBytes);
+                uint8_t* dst = smem + s * kGmStageBytes;
+#pragma unroll
+                for (int bx = 0; bx < 8; ++bx)   // x = (8 ch + bx) * 32 words: a multiple of 128 bytes
+                    tma_load_2d(dst + bx * kGmBoxBytes, &tmap, &full_bar[s], (8 * ch + bx) * 32, b * kGmRows);
             }
             issued = t - t0 + 1;
             if (++s == stages) { s = 0; ph ^= 1u; }
@@ -194,142 +227,108 @@ w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tmap, const GemvParams p) 
         // no copy may still be landing when the CTA exits
         if (lane == 0)
             for (int i = (issued > stages ? issued - stages : 0); i < issued; ++i)
-                mbar_wait(&full_bar[i % stages], static_cast<uint32_t>(i / stages) & 1u, nullptr, kGvDrainLimitNs);
+                mbar_wait(&full_bar[i % stages], static_cast<uint32_t>(i / stages) & 1u, nullptr, kGmDrainLimitNs);
         return;
     }
 
     // -------------------------------------------------------------- consumers
-    // stage x once, token-major, into swizzled 16-byte slots
-    if (XF32) {
-        const int per_tok = C >> 2;                  // 4 columns per unit
-        for (int u = threadIdx.x; u < MT * per_tok; u += 32 * kGvConsumerWarps) {
-            const int m = u / per_tok, c = (u - m * per_tok) << 2;
-            const uint2 v = __ldg(reinterpret_cast<const uint2*>(p.x + static_cast<int64_t>(m) * C + c));
-            const float4 f = make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xFFFF0000u),
-                                         __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xFFFF0000u));
-            *reinterpret_cast<float4*>(xs + static_cast<size_t>(m) * C * 4 + gv_xslot_f32(c >> 5, (c >> 2) & 7)) = f;
+    // stage x once: token m's word w (columns 8w..8w+7) in the order 0,4,1,5,2,6,3,7; columns
+    // past C are zero
+    {
+        const int words = (p.xstride - 64) / 16;
+        for (int u = threadIdx.x; u < p.MT * words; u += 32 * kGmWarps) {
+            const int m = u / words, w = u - m * words;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (w * 8 < p.C) v = __ldg(reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * p.C + w * 8));
+            const uint4 o = make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632),
+                                       __byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
+            *reinterpret_cast<uint4*>(smem + (xs - ring) + m * p.xstride + w * 16) = o;
         }
-    } else {
-        const int per_tok = C >> 3;                  // 8 columns per unit
-        for (int u = threadIdx.x; u < MT * per_tok; u += 32 * kGvConsumerWarps) {
-            const int m = u / per_tok, c = (u - m * per_tok) << 3;
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m) * C + c));
-            *reinterpret_cast<uint4*>(xs + static_cast<size_t>(m) * C * 2 + gv_xslot_bf16(c >> 5, (c >> 3) & 3)) = v;
-        }
+        asm volatile("bar.sync 1, %0;" :: "n"(32 * kGmWarps) : "memory");
     }
-    asm volatile("bar.sync 1, %0;" :: "n"(32 * kGvConsumerWarps) : "memory");
 
-    GvDec dec;
+    const int g = lane >> 2, t = lane & 3;
+    const uint32_t dm = p.dmask, dc = p.dbits;
+    GmScaleCtx sc;
+    sc.scales = p.scales;
+    sc.R = p.R;
+    sc.C = p.C;
+    sc.G = p.G;
+    sc.group = p.group;
+    sc.warp = warp;
+    sc.g = g;
+    sc.fast32 = p.group == 32 && (p.G & 7) == 0;
+    const int R = p.R, MT = p.MT;
+    float* const y = p.y;
+    const bool xtok = g < p.MT;
+    const uint32_t xrow = xs + static_cast<uint32_t>(xtok ? g : 0) * p.xstride + 16u * t;
+    // this lane's word in the codes of rows g and g+8 (the 128-byte swizzle puts chunk k of row r
+    // at (k ^ (r & 7)) * 16; rows g and g+8 share r & 7)
+    uint32_t aoff[kGmQuads];
 #pragma unroll
-    for (int k = 0; k < 5; ++k) {
-        dec.m[k] = p.dmask[k];
-        dec.c[k] = p.dbits[k];
+    for (int j = 0; j < kGmQuads; ++j) {
+        const int q = kGmQuads * warp + j, bx = q >> 3, qq = q & 7;
+        aoff[j] = bx * kGmBoxBytes + g * 128 + ((qq ^ g) << 4) + 4 * t;
     }
-    const int nquads = C >> 5;
-    const int row0 = warp * RPW;                     // first row of this warp in a block
-    const size_t xrow = static_cast<size_t>(C) * XB;
-    // x slots of this lane's quad, relative to the chunk's first quad (a multiple of 32)
-    constexpr int NSLOT = XF32 ? 8 : 4;
-    uint32_t xoff[NSLOT];
-#pragma unroll
-    for (int j = 0; j < NSLOT; ++j) xoff[j] = XF32 ? gv_xslot_f32(lane, j) : gv_xslot_bf16(lane, j);
-    const uint8_t* st_lane = ring + static_cast<size_t>(row0) * kGvRowBytes + 16 * lane;
 
-    float acc[RPW][MT];
-    float s_cur[RPW], s_next[RPW];
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    float s_cur[2 * kGmQuads], s_next[2 * kGmQuads];
     int s = 0, b = b0, ch = ch0;
     uint32_t ph = 0;
-    if (t0 < t1) gv_scales<RPW>(p.scales, R, G, C, group, b, ch, row0, lane, s_next);
-    for (int t = t0; t < t1; ++t) {
-        if (ch == 0 || t == t0) {
+    bool dead = false;   // a bounded wait gave up: skip the work, keep every warp on the same barriers
+    if (t0 < t1) gm_scales(sc, b, ch, s_next);
+    for (int it = t0; it < t1; ++it) {
 #pragma unroll
-            for (int r = 0; r < RPW; ++r)
+        for (int j = 0; j < 2 * kGmQuads; ++j) s_cur[j] = s_next[j];
+        dead = dead || !mbar_wait(&full_bar[s], ph, abort, p.limit_ns);
+        const bool live = !dead;
+        const uint32_t sb = ring + s * kGmStageBytes;
+        uint32_t wa[kGmQuads], wb[kGmQuads];
 #pragma unroll
-                for (int m = 0; m < MT; ++m) acc[r][m] = 0.0f;
+        for (int j = 0; j < kGmQuads; ++j) {
+            wa[j] = live ? gm_lds32(sb + aoff[j]) : 0u;
+            wb[j] = live ? gm_lds32(sb + aoff[j] + 8 * 128) : 0u;
         }
-#pragma unroll
-        for (int r = 0; r < RPW; ++r) s_cur[r] = s_next[r];
-        if (!mbar_wait(&full_bar[s], ph, abort, p.limit_ns)) break;
-        const uint8_t* st = st_lane + static_cast<size_t>(s) * SB;
-        uint4 wq[RPW];
-#pragma unroll
-        for (int r = 0; r < RPW; ++r) wq[r] = *reinterpret_cast<const uint4*>(st + r * kGvRowBytes);
         const int bn = ch + 1 == nchunks ? b + 1 : b, chn = ch + 1 == nchunks ? 0 : ch + 1;
-        if (t + 1 < t1) gv_scales<RPW>(p.scales, R, G, C, group, bn, chn, row0, lane, s_next);
-
-        if (ch * (kGvChunkCols / 32) + lane < nquads) {
-            // the chunk's first quad is 32 * ch: swizzle bits of the lane's quad are the lane's
-            const uint8_t* xq = xs + static_cast<size_t>(ch) * 32 * (32 * XB);
-            float2 part[RPW][MT];
+        if (it + 1 < t1) gm_scales(sc, bn, chn, s_next);
 #pragma unroll
-            for (int r = 0; r < RPW; ++r)
-#pragma unroll
-                for (int m = 0; m < MT; ++m) part[r][m] = make_float2(0.0f, 0.0f);
-#pragma unroll
-            for (int wd = 0; wd < 4; ++wd) {
-                float2 xv[MT][4];               // x of the word's 8 columns, as 4 pairs
-#pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    if (XF32) {
-                        const float4 a = *reinterpret_cast<const float4*>(xq + m * xrow + xoff[2 * wd]);
-                        const float4 c = *reinterpret_cast<const float4*>(xq + m * xrow + xoff[(2 * wd + 1) % NSLOT]);
-                        xv[m][0] = make_float2(a.x, a.y);
-                        xv[m][1] = make_float2(a.z, a.w);
-                        xv[m][2] = make_float2(c.x, c.y);
-                        xv[m][3] = make_float2(c.z, c.w);
-                    } else {
-                        const uint4 xr = *reinterpret_cast<const uint4*>(xq + m * xrow + xoff[wd % NSLOT]);
-                        xv[m][0] = make_float2(__uint_as_float(xr.x << 16), __uint_as_float(xr.x & 0xFFFF0000u));
-                        xv[m][1] = make_float2(__uint_as_float(xr.y << 16), __uint_as_float(xr.y & 0xFFFF0000u));
-                        xv[m][2] = make_float2(__uint_as_float(xr.z << 16), __uint_as_float(xr.z & 0xFFFF0000u));
-                        xv[m][3] = make_float2(__uint_as_float(xr.w << 16), __uint_as_float(xr.w & 0xFFFF0000u));
-                    }
-                }
-#pragma unroll
-                for (int r = 0; r < RPW; ++r) {
-                    const uint32_t word = wd == 0 ? wq[r].x : wd == 1 ? wq[r].y : wd == 2 ? wq[r].z : wq[r].w;
-                    float2 v[4];
-                    gv_decode(word, dec, v);
-#pragma unroll
-                    for (int m = 0; m < MT; ++m) {
-                        part[r][m] = __ffma2_rn(xv[m][0], v[0], part[r][m]);
-                        part[r][m] = __ffma2_rn(xv[m][1], v[1], part[r][m]);
-                        part[r][m] = __ffma2_rn(xv[m][2], v[2], part[r][m]);
-                        part[r][m] = __ffma2_rn(xv[m][3], v[3], part[r][m]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int r = 0; r < RPW; ++r)
-#pragma unroll
-                for (int m = 0; m < MT; ++m) acc[r][m] = fmaf(s_cur[r], part[r][m].x + part[r][m].y, acc[r][m]);
+        for (int j = 0; live && j < kGmQuads; ++j) {
+            const int q = ch * (kGmChunkCols / 32) + kGmQuads * warp + j;   // group of 32 in the row
+            uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+            if (xtok) xv = gm_lds128(xrow + q * 64);
+            float d[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            gm_mma(d, gm_pair(wa[j], dm, dc), gm_pair(wb[j], dm, dc), gm_pair(wa[j] >> 4, dm, dc),
+                   gm_pair(wb[j] >> 4, dm, dc), xv.x, xv.y);
+            gm_mma(d, gm_pair(wa[j] >> 8, dm, dc), gm_pair(wb[j] >> 8, dm, dc), gm_pair(wa[j] >> 12, dm, dc),
+                   gm_pair(wb[j] >> 12, dm, dc), xv.z, xv.w);
+            acc[0] = fmaf(s_cur[2 * j], d[0], acc[0]);
+            acc[1] = fmaf(s_cur[2 * j], d[1], acc[1]);
+            acc[2] = fmaf(s_cur[2 * j + 1], d[2], acc[2]);
+            acc[3] = fmaf(s_cur[2 * j + 1], d[3], acc[3]);
         }
         // the slot is released only once the codes loaded from it have been used: a release
         // issued while a shared load is still in flight does not keep the next bulk copy from
         // overwriting the slot under it
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[s]);
+        if (lane == 0 && live) mbar_arrive(&empty_bar[s]);
 
-        if (ch == nchunks - 1 || t == t1 - 1) {
+        if (ch == nchunks - 1 || it == t1 - 1) {
+            // the eight warps' partial tiles, summed in warp order
 #pragma unroll
-            for (int r = 0; r < RPW; ++r)
+            for (int c = 0; c < 4; ++c) red[(warp * 32 + lane) * 4 + c] = acc[c];
+            asm volatile("bar.sync 1, %0;" :: "n"(32 * kGmWarps) : "memory");
+            if (threadIdx.x < 128) {
+                const int ol = threadIdx.x >> 2, oc = threadIdx.x & 3;      // output of lane ol, entry oc
+                float v = 0.0f;
 #pragma unroll
-                for (int m = 0; m < MT; ++m) {
-                    float v = acc[r][m];
-#pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-                    acc[r][m] = v;
-                }
-            if (lane == 0) {
-#pragma unroll
-                for (int r = 0; r < RPW; ++r) {
-                    const int row = b * RB + row0 + r;
-                    if (row < R) {
-#pragma unroll
-                        for (int m = 0; m < MT; ++m) atomicAdd(p.y + static_cast<int64_t>(m) * R + row, acc[r][m]);
-                    }
-                }
+                for (int w = 0; w < kGmWarps; ++w) v += red[(w * 32 + ol) * 4 + oc];
+                const int row = b * kGmRows + (ol >> 2) + (oc >= 2 ? 8 : 0);
+                const int tok = 2 * (ol & 3) + (oc & 1);
+                if (row < R && tok < MT && !*abort) atomicAdd(y + static_cast<int64_t>(tok) * R + row, v);
             }
+            asm volatile("bar.sync 1, %0;" :: "n"(32 * kGmWarps) : "memory");
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[c] = 0.0f;
         }
         if (++s == stages) {
             s = 0;

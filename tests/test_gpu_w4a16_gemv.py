@@ -45,9 +45,11 @@ def _check(W, D, M, oracle_mod, rowwise=False):
 
 
 @pytest.mark.parametrize("R,C,M", [(1, 32, 1), (33, 96, 2), (70, 2080, 3), (64, 4096, 4), (45, 32 * 129, 5),
-                                   (31, 14336, 1), (50, 30016, 4)])
+                                   (31, 14336, 1), (50, 30016, 4), (100, 4096, 8), (17, 1056, 9),
+                                   (300, 14336, 7)])
 def test_gemv_group32(R, C, M, oracle_mod):
-    """Ragged rows and columns, 1..5 tokens; C = 30016 leaves room for 3 tokens per pass only."""
+    """Ragged rows and columns, 1..9 tokens (more than 8 take two passes); C = 30016 leaves room
+    for 3 tokens per pass only, C = 14336 for 6."""
     _check(*_export(R, C, seed=R * 7 + C), M, oracle_mod)
 
 
