@@ -114,10 +114,12 @@ qat4_status qat4_hessian_partial(const uint16_t *X, int64_t n, int64_t C, int64_
  *  idx       out int32   [R, C/32]: the chosen k (smallest k on exact ties).
  *  best_err  out float32 [R, C/32] (may be NULL): e H_gg e^T at the chosen k,
  *            rounded to float32 from a float64 evaluation.
- *  Every candidate is screened in float32 with a rigorous rounding-error
- *  bound; the candidates that the bound cannot separate from the minimum
- *  are re-scored in float64, so idx equals the argmin of the float64
- *  objective except for candidates whose objectives agree to ~1e-15.
+ *  Every candidate is screened on the tensor cores (e H e^T with the error
+ *  vector in binary16 and H split into two binary16 parts, float32 sums)
+ *  together with a rigorous rounding-error bound; the candidates that the
+ *  bound cannot separate from the minimum are re-scored in float64, so idx
+ *  equals the argmin of the float64 objective except for candidates whose
+ *  objectives agree to ~1e-15.
  *  Errors: QAT4_ERR_NULL, _SHAPE, _ALIGN, _CUDA.
  */
 qat4_status qat4_scale_search(const float *W, int64_t R, int64_t C,

@@ -75,19 +75,6 @@ constexpr uint32_t kFqIdesc = (1u << 4)            // D format: F32
                             | ((256u >> 3) << 17)  // N >> 3
                             | ((256u >> 4) << 24); // M >> 4
 
-// Shared-memory descriptor of a K-major operand in the 128-byte swizzle layout: rows of 128 B,
-// 8-row groups 1 KB apart (stride byte offset); the leading byte offset is unused for a
-// swizzled K-major operand whose K extent is one swizzle row.
-__device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t saddr) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>(1) << 16;
-    d |= static_cast<uint64_t>((1024u >> 4) & 0x3FFFu) << 32;
-    d |= static_cast<uint64_t>(1) << 46;   // descriptor version (sm_100)
-    d |= static_cast<uint64_t>(2) << 61;   // SWIZZLE_128B
-    return d;
-}
-
 struct FqParams {
     const float* delta;   // [R, C/32]
     float* Y;             // [T, R]

@@ -211,16 +211,16 @@ qat4_status qat4_scale_search(const float* W, int64_t R, int64_t C, const float*
     {
         std::lock_guard<std::mutex> lock(g_mutex);
         if (!info->search_attr) {
-            if (cudaFuncSetAttribute(qat4::scale_search_kernel<3, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(sizeof(qat4::SearchSmem))) != cudaSuccess)
+            if (cudaFuncSetAttribute(qat4::scale_search_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(qat4::kTcSmemBytes)) != cudaSuccess)
                 return QAT4_ERR_CUDA;
             info->search_attr = true;
         }
     }
-    const dim3 grid(static_cast<unsigned>((R + qat4::kSearchThreads - 1) / qat4::kSearchThreads),
-                    static_cast<unsigned>(C / 32));
-    qat4::scale_search_kernel<3, 1><<<grid, qat4::kSearchThreads, sizeof(qat4::SearchSmem), stream>>>(
-        W, static_cast<int>(R), static_cast<int>(C), H, ldh, alpha, K, delta, idx, best_err);
+    const dim3 grid(static_cast<unsigned>((R + qat4::kTcRows - 1) / qat4::kTcRows), static_cast<unsigned>(C / 32));
+    // each wait covers one candidate's four small MMAs; the limit only catches a tensor core that never answers
+    qat4::scale_search_kernel<4><<<grid, qat4::kTcRows, qat4::kTcSmemBytes, stream>>>(
+        W, static_cast<int>(R), static_cast<int>(C), H, ldh, alpha, K, delta, idx, best_err, 4000000000ull);
     return launch_status();
 }
 

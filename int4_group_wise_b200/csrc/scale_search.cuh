@@ -1,222 +1,62 @@
-// scale_search.cuh -- Hessian-weighted per-group scale search.
+// scale_search.cuh -- the Hessian-weighted per-group scale search with the
+// quadratic forms on the 5th-generation tensor cores.
 //
 // Model card "Opt.Gear-1B-qat-int4-per-channel-unquantized", section
-// "Quantization Configuration": the scale of every quantization group is
-// initialised by minimising the layer-output reconstruction error
-// ||W X - Q_Delta(W) X||^2.  Read block-diagonally, group (r, g) minimises
-// E(Delta) = e H_gg e^T with e = w_g - Q_Delta(w_g) and H_gg the 32x32 diagonal
-// block of H, over the candidates Delta_k = fl(alpha_k * fl(max|w_g| / 7)).
+// "Quantization Configuration": the scale of every group minimises the
+// layer-output error ||W X - Q_Delta(W) X||^2; read block-diagonally, group
+// (r, g) minimises E_k = e H_gg e^T over the candidates
+// Delta_k = fl(alpha_k * fl(max|w_g| / 7)), with e = w - fl(Delta_k q) the
+// exact difference of the binary32 weights and their quantized values.
 //
-// The error vector is the exact difference e = w - Q_Delta(w) of the binary32
-// weights and their binary32 quantized values.
+// Mapping: one CTA = one column group g x 128 rows (thread = row = TMEM lane =
+// row of the MMA's M = 128 tile).  For every candidate k the 128 threads
+// quantize their 32 weights (exact codes, see tc_quantize) and write
+// the error vector e as binary16 e_hi into the A operand in shared memory; one
+// thread issues tcgen05.mma.kind::f16 (M = 128, N = 32, K = 16):
+//     P = e_hi * (H_hi + H_lo)        (float32 accumulate in TMEM)
+// where H_hi + H_lo is the symmetrised block (H + H^T)/2, scaled by a power of
+// two into binary16 range and split into two binary16 parts.  Each thread then
+// reads its row of P back and forms E = P . v, v = e + e_lo = 2e - e_hi: since
+// e = e_hi + e_lo exactly and H is symmetric,
+//     e H e = e_hi H (e + e_lo) + e_lo H e_lo,
+// so one binary16 A operand gives E to about 2^-22 relative (the dropped
+// e_lo H e_lo term is <= 2^-22 of the form's scale).  Weights are scaled by
+// a power of two per row (2^13 <= max|w| sigma < 2^14) so that e fits binary16
+// without overflow; scaling by powers of two leaves the codes and the argmin
+// unchanged.
 //
-// Mapping: one CTA = one column group g x 128 rows; thread t owns row
-// r0 + t and keeps its 32 weights in registers.  H_gg is staged once per CTA
-// in shared memory as the upper triangle of H'_{ij} = H_ij + H_ji (j > i),
-// H'_ii = H_ii (528 floats, stored twice and read as broadcast float4), so
-// that E = sum_i e_i * (sum_{j >= i} H'_ij e_j): 528 + 32 FMA per candidate.
-// Each thread evaluates two candidates per pass with packed FP32x2
-// instructions (one FFMA2 = one FMA of each candidate); the quantization
-// steps are packed the same way.
+// Two-stage pipeline: while the tensor core multiplies candidate k, the
+// threads quantize candidate k + 1.  Each thread parks its v of a candidate in
+// TMEM next to that candidate's P (columns 64s..64s+31 hold P of stage s,
+// 64s+32..64s+63 hold v), so the pipeline costs no registers and four CTAs
+// fit on an SM; the two stages' A operands share each 128-byte row (bytes
+// 64s..64s+63).  One CTA barrier per candidate hands the A stage to the
+// tensor core; the issuing thread rotates over the four warps.
 //
-// Exactness: the codes are exact (rint of the IEEE quotient w / Delta_k; the
-// quotient is formed as w * (1/Delta_k) and the IEEE division is redone for
-// the group whenever that product lands within 2^-18 of a rounding boundary,
-// which a 3-ulp error analysis shows is the only place the two can differ).
-// E is screened in float32 together with a rigorous bound
-//     |E32 - E| <= 80 u kappa S^2,   S = sum_i |e_i| sqrt|H_ii|,  u = 2^-24,
-// kappa = max(1, max_{i != j} |H_ij| / sqrt|H_ii H_jj|)  (= 1 for a PSD H)
-// which covers the <= 33-term FMA sums (about 66u), the rounding of H' and of
-// the float32 difference fl(w - Q) used by the screen (about 3u).  Every candidate
-// whose interval [E32 - b, E32 + b] can still contain the minimum is
-// re-scored in float64 (the top four lower bounds are kept; if four or more
-// are undecided, all K candidates are re-scored), and the float64 minimum
-// wins, smallest k on ties.
+// The screened value carries a rigorous bound
+//     |E_screen - E| <= c * Sa^2 + c_f * T * Sa,
+//     Sa = (1 + 2^-9)(S + 2^-14 T),  S = sum_i |v_i| sd_i,  T = sum_i sd_i,
+//     sd_i = sqrt|H_ii| (scaled, rounded up),
+//     c = (kappa + kappa_d)(tau + 2^-19 + 2^-22) + kappa_d + kappa (2^-20 + 2^-23),
+// with kappa = max(1, max_{i != j} |H_ij| / (sd_i sd_j)), kappa_d the same ratio
+// for the error of the binary16 split of H (computed exactly per CTA), tau =
+// 2^-17 covering 64 float32 accumulation steps of the tensor core at one unit
+// in the last place each (products of binary16 values are exact in float32),
+// and c_f = 2^-12 (kappa + kappa_d) covering a tensor core that would flush
+// binary16 subnormal inputs (e_hi < 2^-14) to zero.  Candidates whose
+// interval can still hold the minimum are re-scored in float64
+// (tc_quad_form64), so the returned index is the float64 argmin.
 #pragma once
 
-#include <cstddef>
-#include <utility>
+#include <cuda_fp16.h>
 
 #include "device_common.cuh"
 
 namespace qat4 {
 
-constexpr int kSearchThreads = 128;
 constexpr int kTri = 528;          // entries of the upper triangle of a 32x32 block
 constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23: x + M - M = rint(x) for |x| < 2^22
 constexpr float kTieWindow = 0.5f - 3.814697265625e-06f;  // 0.5 - 2^-18
-constexpr float kBoundC = 80.0f * 5.9604644775390625e-08f;  // 80 * 2^-24
-
-// Row / column of entry p of the row-major upper triangle (j >= i) of a 32x32 matrix.
-__host__ __device__ constexpr int tri_row(int p) {
-    int i = 0;
-    while (p >= 32 - i) { p -= 32 - i; ++i; }
-    return i;
-}
-__host__ __device__ constexpr int tri_col(int p) {
-    int i = 0;
-    while (p >= 32 - i) { p -= 32 - i; ++i; }
-    return i + p;
-}
-static_assert(tri_row(527) == 31 && tri_col(527) == 31 && tri_col(31) == 31 && tri_row(32) == 1, "tri");
-
-constexpr int kSlot = 36;          // floats per thread slot (144 B: float4-aligned, few bank conflicts)
-
-struct SearchSmem {
-    float4 h32[kTri / 2];   // H' upper triangle, float32, each entry twice: (h_p, h_p, h_p+1, h_p+1)
-    double h64[kTri];       // same, float64 (H_ij + H_ji exact)
-    float4 sqrt_diag[8];    // sqrt(|H_ii|), rounded up
-    float hfull[32][33];    // staging copy of H_gg (padded)
-    unsigned kappa_bits;    // kappa as float bits (non-negative: int order == float order)
-    // per-thread copies of the 32 weights and of an error vector, used only by
-    // the exact (IEEE division) path so that it stays out of the unrolled loop
-    alignas(16) float wslot[kSearchThreads * kSlot];
-    alignas(16) float eslot[kSearchThreads * kSlot];
-};
-// every float4 access below needs these offsets to be multiples of 16 bytes
-static_assert(sizeof(float4) * (kTri / 2) == 2 * kTri * sizeof(float) && offsetof(SearchSmem, h32) % 16 == 0 && offsetof(SearchSmem, sqrt_diag) % 16 == 0 &&
-              offsetof(SearchSmem, h64) % 8 == 0 && offsetof(SearchSmem, wslot) % 16 == 0 &&
-              offsetof(SearchSmem, eslot) % 16 == 0 && (kSlot * 4) % 16 == 0, "SearchSmem alignment");
-
-// Exact error vector of one candidate from the weights parked in shared
-// memory: q = clamp(rint(w / dk), -8, 7) with the IEEE division, in a rolled
-// loop (taken only near a rounding boundary or when 1/dk is not finite).
-__device__ __noinline__ void group_error_exact(const float* wslot, float dk, float* eslot) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i) {
-        const float wi = wslot[i];
-        const float q = code_of(scaled_exact(wi, dk));
-        eslot[i] = __fsub_rn(wi, __fmul_rn(dk, q));
-    }
-}
-
-// e_i = fl(w_i - fl(dk * q_i)), q_i = clamp(rint(fl(w_i / dk)), -8, 7).
-// wslot / eslot: this thread's shared-memory slots (wslot holds w).
-__device__ __forceinline__ void group_error(const float (&w)[32], float dk, float (&e)[32],
-                                            const float* wslot, float* eslot) {
-    const float rc = __frcp_rn(dk);
-    bool slow = !(fabsf(rc) <= 3.4028234663852886e38f);   // dk == 0 or 1/dk overflows
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const float r = fminf(fmaxf(__fmul_rn(w[i], rc), kQmin), kQmax);
-        const float q = __fsub_rn(__fadd_rn(r, kMagic), kMagic);
-        slow |= !(fabsf(__fsub_rn(r, q)) <= kTieWindow);
-        e[i] = __fsub_rn(w[i], __fmul_rn(dk, q));
-    }
-    if (slow) {
-        group_error_exact(wslot, dk, eslot);
-        const float4* e4 = reinterpret_cast<const float4*>(eslot);
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-            const float4 x = e4[v];
-            e[4 * v] = x.x; e[4 * v + 1] = x.y; e[4 * v + 2] = x.z; e[4 * v + 3] = x.w;
-        }
-    }
-}
-
-// Two candidates at once: element j of the pair register holds (e0_j, e1_j);
-// one packed FMA (FFMA2) advances both candidates' row sums.  Each row sum is
-// split into NCH interleaved chains (j - i mod NCH) so consecutive FFMA2s do
-// not wait on each other; the chains are added at the end of the row.  (The
-// screening bound holds for any summation order of these <= 33-term sums.)
-template <int NCH, int P>
-__device__ __forceinline__ void tri_ffma2(float2 h, const float2 (&e)[32], float2 (&t)[NCH], float2& E) {
-    constexpr int i = tri_row(P);
-    constexpr int j = tri_col(P);
-    constexpr int c = (j - i) % NCH;
-    t[c] = __ffma2_rn(h, e[j], t[c]);
-    if constexpr (j == 31) {
-        float2 r = t[0];
-#pragma unroll
-        for (int x = 1; x < NCH; ++x) r = __fadd2_rn(r, t[x]);
-        E = __ffma2_rn(e[i], r, E);
-#pragma unroll
-        for (int x = 0; x < NCH; ++x) t[x] = make_float2(0.0f, 0.0f);
-    }
-}
-
-template <int NCH, int Q2>
-__device__ __forceinline__ void tri_pair2(const float4* h32, const float2 (&e)[32], float2 (&t)[NCH], float2& E) {
-    const float4 h = h32[Q2];                     // (h_p, h_p, h_p+1, h_p+1)
-    tri_ffma2<NCH, 2 * Q2 + 0>(make_float2(h.x, h.y), e, t, E);
-    tri_ffma2<NCH, 2 * Q2 + 1>(make_float2(h.z, h.w), e, t, E);
-}
-
-template <int NCH, int... Q2s>
-__device__ __forceinline__ float2 quad_form_pair_impl(std::integer_sequence<int, Q2s...>, const float4* h32,
-                                                      const float2 (&e)[32]) {
-    float2 t[NCH];
-#pragma unroll
-    for (int x = 0; x < NCH; ++x) t[x] = make_float2(0.0f, 0.0f);
-    float2 E = make_float2(0.0f, 0.0f);
-    (tri_pair2<NCH, Q2s>(h32, e, t, E), ...);
-    return E;
-}
-
-// float32 screening values of two candidates, E.x and E.y.
-template <int NCH>
-__device__ __forceinline__ float2 quad_form_pair(const float4* h32, const float2 (&e)[32]) {
-    return quad_form_pair_impl<NCH>(std::make_integer_sequence<int, kTri / 2>{}, h32, e);
-}
-
-// Error vectors of two candidates (dk.x, dk.y) in packed form; every
-// component goes through exactly the operations of group_error, so the
-// values are bit-identical to it.
-__device__ __forceinline__ void group_error_pair(const float2 (&w2)[32], float2 dk, float2 (&e)[32],
-                                                 const float* wslot, float* eslot) {
-    const float2 rc = make_float2(__frcp_rn(dk.x), __frcp_rn(dk.y));
-    bool slow = !(fabsf(rc.x) <= 3.4028234663852886e38f) || !(fabsf(rc.y) <= 3.4028234663852886e38f);
-    const float2 M = make_float2(kMagic, kMagic);
-    const float2 negM = make_float2(-kMagic, -kMagic);
-    const float2 neg1 = make_float2(-1.0f, -1.0f);
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        float2 r = __fmul2_rn(w2[i], rc);
-        r.x = fminf(fmaxf(r.x, kQmin), kQmax);
-        r.y = fminf(fmaxf(r.y, kQmin), kQmax);
-        const float2 q = __fadd2_rn(__fadd2_rn(r, M), negM);     // rint, exact for |r| <= 8
-        const float2 f = __ffma2_rn(q, neg1, r);                  // r - q
-        slow |= !(fabsf(f.x) <= kTieWindow) || !(fabsf(f.y) <= kTieWindow);
-        e[i] = __ffma2_rn(__fmul2_rn(dk, q), neg1, w2[i]);       // w - fl(dk * q)
-    }
-    if (slow) {
-        const float4* e4 = reinterpret_cast<const float4*>(eslot);
-        group_error_exact(wslot, dk.x, eslot);
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-            const float4 x = e4[v];
-            e[4 * v].x = x.x; e[4 * v + 1].x = x.y; e[4 * v + 2].x = x.z; e[4 * v + 3].x = x.w;
-        }
-        group_error_exact(wslot, dk.y, eslot);
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-            const float4 x = e4[v];
-            e[4 * v].y = x.x; e[4 * v + 1].y = x.y; e[4 * v + 2].y = x.z; e[4 * v + 3].y = x.w;
-        }
-    }
-}
-
-// float64 value of one candidate (the re-score): codes with the IEEE
-// division, Q = fl(dk * q), and the exact difference e = w - Q (exact in
-// binary64), summed in binary64.
-__device__ __forceinline__ double quad_form64(const double* h64, const float (&w)[32], float dk) {
-    double ed[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        const float q = code_of(scaled_exact(w[i], dk));
-        ed[i] = static_cast<double>(w[i]) - static_cast<double>(__fmul_rn(dk, q));
-    }
-    double E = 0.0;
-    int p = 0;
-#pragma unroll
-    for (int i = 0; i < 32; ++i) {
-        double t = 0.0;
-#pragma unroll
-        for (int j = i; j < 32; ++j) t = fma(h64[p++], ed[j], t);
-        E = fma(ed[i], t, E);
-    }
-    return E;
-}
 
 struct TopK4 {
     float L[4];
@@ -239,133 +79,483 @@ struct TopK4 {
     }
 };
 
-template <int MINB, int NCH>
-__global__ void __launch_bounds__(kSearchThreads, MINB)
+constexpr int kTcRows = 128;
+constexpr int kTcSlot = 36;                      // floats per exact-path slot
+// kind::f16 instruction descriptor: D float32, A and B binary16, both K-major, N = 32, M = 128.
+constexpr uint32_t kTcIdesc = (1u << 4) | ((32u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t kTcStageCols = 64;            // TMEM columns per stage: P (32) then v (32)
+constexpr uint32_t kTcTmemCols = 2 * kTcStageCols;
+
+struct SearchTcSmem {
+    // A: row m holds thread m's e_hi (binary16) of stage 0 in bytes 0..63 and of
+    // stage 1 in bytes 64..127 (K-major, 128-byte swizzle)
+    uint8_t a[kTcRows * 128];
+    uint8_t bhi[32 * 128];        // row n: column n of the scaled symmetrised block, hi part (k < 32)
+    uint8_t blo[32 * 128];        //        the lo part
+    double h64[kTri];             // H'_ij = H_ij + H_ji (j > i), H'_ii = H_ii, binary64, unscaled
+    union {
+        float hfull[32][33];                       // set-up: staging copy of H_gg
+        float eslot[kTcRows * kTcSlot];            // main loop: exact-path error vectors
+    } u;
+    uint64_t mbar[2];
+    uint32_t tmem_base;
+    unsigned kappa_bits;          // kappa (non-negative float bits)
+    unsigned kappa_d_bits;        // kappa_d
+    unsigned hmax_bits;           // max |H_sym| (unscaled)
+    int exact_block;              // the split cannot represent this block: re-score every candidate
+    int abort;
+    float coef, coef_f, tsum;
+    alignas(16) float sd[32];     // sqrt(sigma_H |H_ii|), rounded up
+    float isd[32];                // reciprocals rounded up (set-up only)
+};
+constexpr size_t kTcSmemBytes = sizeof(SearchTcSmem) + 1024;   // + alignment of the operand tiles
+static_assert(offsetof(SearchTcSmem, a) == 0 && offsetof(SearchTcSmem, bhi) % 1024 == 0 &&
+              offsetof(SearchTcSmem, blo) % 1024 == 0 && offsetof(SearchTcSmem, u) % 16 == 0 &&
+              offsetof(SearchTcSmem, mbar) % 8 == 0 && offsetof(SearchTcSmem, sd) % 16 == 0,
+              "SearchTcSmem layout");
+
+// Byte offset of logical 16-byte chunk c of row n in a K-major 128-byte-swizzled tile.
+__host__ __device__ constexpr uint32_t sw128_off(uint32_t n, uint32_t c) {
+    return n * 128u + ((c ^ (n & 7u)) << 4);
+}
+
+// Round-up helper for the bound (non-negative inputs).
+__device__ __forceinline__ float up(double x) { return __double2float_ru(x); }
+
+// Exact error vector of one candidate, scaled: e_i = sigma * fl(w_i - fl(dk * q_i)),
+// q_i = clamp(rint(fl(w_i / dk)), -8, 7) with the IEEE division; w read from global
+// memory (rolled loop, taken only near a rounding boundary or when 1/dk is not finite).
+__device__ __noinline__ void tc_error_exact(const float* __restrict__ wrow, float dk, float sigma, float* eslot) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i) {
+        const float wi = wrow[i];
+        const float q = code_of(scaled_exact(wi, dk));
+        eslot[i] = __fmul_rn(__fsub_rn(wi, __fmul_rn(dk, q)), sigma);
+    }
+}
+
+// Start of row i of the row-major upper triangle (j >= i) of a 32x32 matrix.
+__host__ __device__ constexpr int tri_start(int i) { return 32 * i - (i * (i - 1)) / 2; }
+
+// float64 value of one candidate (the re-score): codes with the IEEE division,
+// Q = fl(dk * q), the exact difference e = w - Q (exact in binary64), and
+// e H' e summed in binary64 over the upper triangle H' (H'_ij = H_ij + H_ji,
+// H'_ii = H_ii).  Two rows at a time, each row's sum split in two, so four
+// independent FMA chains are in flight.
+__device__ __forceinline__ double tc_quad_form64(const double* h64, const float (&w)[32], float dk) {
+    double ed[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const float q = code_of(scaled_exact(w[i], dk));
+        ed[i] = static_cast<double>(w[i]) - static_cast<double>(__fmul_rn(dk, q));
+    }
+    double E0 = 0.0, E1 = 0.0;
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        double ta = 0.0, tb = 0.0, tc = 0.0, td = 0.0;
+        const double* ra = h64 + tri_start(i);          // row i: j = i..31
+        const double* rb = h64 + tri_start(i + 1);      // row i + 1: j = i + 1..31
+#pragma unroll
+        for (int j = i; j < 32; ++j) {
+            if ((j - i) & 1) tb = fma(ra[j - i], ed[j], tb);
+            else ta = fma(ra[j - i], ed[j], ta);
+        }
+#pragma unroll
+        for (int j = i + 1; j < 32; ++j) {
+            if ((j - i - 1) & 1) td = fma(rb[j - i - 1], ed[j], td);
+            else tc = fma(rb[j - i - 1], ed[j], tc);
+        }
+        E0 = fma(ed[i], ta + tb, E0);
+        E1 = fma(ed[i + 1], tc + td, E1);
+    }
+    return E0 + E1;
+}
+
+// Quantizes one candidate for this thread's row: writes e_hi into the stage's
+// half of its A row, parks v = 2e - e_hi in the stage's TMEM columns (this
+// thread's lane) and returns S = sum |v_i| sd_i.
+__device__ __forceinline__ float tc_quantize(const float2 (&ws)[16], float dk, float sig, bool screen,
+                                             const float* __restrict__ wrow, float* eslot, const float* sd,
+                                             uint32_t a_row, uint32_t swz, uint32_t stage, uint32_t tv) {
+    const float ds = __fmul_rn(dk, sig);                              // scaled (exact power of two)
+    const float rc = __frcp_rn(ds);
+    const float2 d2 = make_float2(ds, ds);
+    const float2 rc2 = make_float2(rc, rc);
+    const float2 M2 = make_float2(kMagic, kMagic);
+    const float2 negM2 = make_float2(-kMagic, -kMagic);
+    const float2 neg1 = make_float2(-1.0f, -1.0f);
+    float2 v[16];
+    float fmax_abs = 0.0f;                                            // max_i |x_i - q_i|
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        float2 x = __fmul2_rn(ws[j], rc2);
+        x.x = fminf(fmaxf(x.x, kQmin), kQmax);
+        x.y = fminf(fmaxf(x.y, kQmin), kQmax);
+        const float2 q = __fadd2_rn(__fadd2_rn(x, M2), negM2);       // rint, exact for |x| <= 8
+        const float2 f = __ffma2_rn(q, neg1, x);                      // x - q
+        fmax_abs = fmaxf(fmax_abs, fmaxf(fabsf(f.x), fabsf(f.y)));
+        v[j] = __ffma2_rn(__fmul2_rn(d2, q), neg1, ws[j]);           // e = w - fl(d q), scaled
+    }
+    // near a rounding boundary (or 1/ds not finite) redo the codes with the IEEE division
+    if (screen && !(fmax_abs <= kTieWindow && fabsf(rc) <= 3.4028234663852886e38f)) {
+        tc_error_exact(wrow, dk, sig, eslot);
+        const float4* e4 = reinterpret_cast<const float4*>(eslot);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float4 x = e4[c];
+            v[2 * c] = make_float2(x.x, x.y);
+            v[2 * c + 1] = make_float2(x.z, x.w);
+        }
+    }
+    const float2 two = make_float2(2.0f, 2.0f);
+    float S0 = 0.0f, S1 = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        uint32_t hw[4];
+        const float4 sa = reinterpret_cast<const float4*>(sd)[2 * c];
+        const float4 sb = reinterpret_cast<const float4*>(sd)[2 * c + 1];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int j = 4 * c + t;
+            const __half2 h = __float22half2_rn(v[j]);
+            const float2 hf = __half22float2(h);
+            v[j] = __ffma2_rn(v[j], two, make_float2(-hf.x, -hf.y));   // v = e + e_lo = 2e - e_hi
+            hw[t] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        S0 = fmaf(fabsf(v[4 * c].x), sa.x, S0);
+        S1 = fmaf(fabsf(v[4 * c].y), sa.y, S1);
+        S0 = fmaf(fabsf(v[4 * c + 1].x), sa.z, S0);
+        S1 = fmaf(fabsf(v[4 * c + 1].y), sa.w, S1);
+        S0 = fmaf(fabsf(v[4 * c + 2].x), sb.x, S0);
+        S1 = fmaf(fabsf(v[4 * c + 2].y), sb.y, S1);
+        S0 = fmaf(fabsf(v[4 * c + 3].x), sb.z, S0);
+        S1 = fmaf(fabsf(v[4 * c + 3].y), sb.w, S1);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                     :: "r"(a_row + (((4u * stage + static_cast<uint32_t>(c)) ^ swz) << 4)),
+                        "r"(hw[0]), "r"(hw[1]), "r"(hw[2]), "r"(hw[3]) : "memory");
+    }
+    uint32_t vb[32];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+        vb[2 * j] = __float_as_uint(v[j].x);
+        vb[2 * j + 1] = __float_as_uint(v[j].y);
+    }
+    tmem_st_32x32b_x32(tv, vb);
+    return S0 + S1;
+}
+
+// The MMAs of one candidate (issued by one thread): P = e_hi (H_hi + H_lo) into
+// the stage's TMEM columns 0..31.
+__device__ __forceinline__ void tc_issue(uint32_t tmem_stage, uint32_t a_stage, uint32_t bh, uint32_t bl,
+                                         uint64_t* bar) {
+    tc_fence_after();
+#pragma unroll
+    for (uint32_t kk = 0; kk < 2; ++kk)
+        tc_mma_f16(tmem_stage, smem_desc_k_sw128(a_stage + 32u * kk), smem_desc_k_sw128(bh + 32u * kk),
+                   kTcIdesc, kk > 0 ? 1u : 0u);
+#pragma unroll
+    for (uint32_t kk = 0; kk < 2; ++kk)
+        tc_mma_f16(tmem_stage, smem_desc_k_sw128(a_stage + 32u * kk), smem_desc_k_sw128(bl + 32u * kk),
+                   kTcIdesc, 1u);
+    tc_commit(bar);
+}
+
+struct TcBound {
+    float coef, coef_f, tsum;
+};
+
+// Reads candidate k's P row and v from TMEM, forms E = P . v and its bound, and
+// records them.  Returns false if the wait for the MMAs gave up.
+__device__ __forceinline__ bool tc_consume(int k, uint32_t tst, uint64_t* bar, volatile int* abort,
+                                           uint64_t limit_ns, float S, const TcBound& tb,
+                                           TopK4& top, float& upper) {
+    if (!mbar_wait_parked(bar, static_cast<uint32_t>((k >> 1) & 1), abort, limit_ns)) return false;
+    tc_fence_after();
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t P[16], V[16];
+        tmem_ld_32x32b_x16(tst + 16u * h, P);
+        tmem_ld_32x32b_x16(tst + 32u + 16u * h, V);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            acc[j & 3] = fmaf(__uint_as_float(P[j]), __uint_as_float(V[j]), acc[j & 3]);
+    }
+    const float E = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    const float Sa = __fmul_ru(1.001953125f, __fmaf_ru(6.103515625e-05f, tb.tsum, S));     // (1+2^-9)(S + 2^-14 T)
+    const float b = __fmaf_ru(tb.coef, __fmul_ru(Sa, Sa), __fmul_ru(tb.coef_f, __fmul_ru(tb.tsum, Sa)));
+    upper = fminf(upper, E + b);
+    top.insert(E - b, k);
+    return true;
+}
+
+template <int MINB>
+__global__ void __launch_bounds__(kTcRows, MINB)
 scale_search_kernel(const float* __restrict__ W, int R, int C,
-                    const float* __restrict__ H, int64_t ldh,
-                    const float* __restrict__ alpha, int K,
-                    float* __restrict__ delta_out, int* __restrict__ idx_out,
-                    float* __restrict__ err_out) {
-    extern __shared__ __align__(16) uint8_t search_smem_raw[];
-    SearchSmem& sm = *reinterpret_cast<SearchSmem*>(search_smem_raw);
+                       const float* __restrict__ H, int64_t ldh,
+                       const float* __restrict__ alpha, int K,
+                       float* __restrict__ delta_out, int* __restrict__ idx_out,
+                       float* __restrict__ err_out, uint64_t limit_ns) {
+    extern __shared__ __align__(16) uint8_t tc_smem_raw[];
+    const uint32_t raw = smem_u32(tc_smem_raw);
+    SearchTcSmem& sm = *reinterpret_cast<SearchTcSmem*>(tc_smem_raw + ((1024u - (raw & 1023u)) & 1023u));
     const int g = blockIdx.y;
     const int G = C / kGroup;
     const int tid = threadIdx.x;
+    const int warp = tid >> 5;
 
-    // ---- stage H_gg and its derived tables
-    const float* Hg = H + static_cast<int64_t>(g) * kGroup * ldh + static_cast<int64_t>(g) * kGroup;
-    for (int x = tid; x < 32 * 32; x += kSearchThreads) {
-        const int i = x >> 5, j = x & 31;
-        sm.hfull[i][j] = Hg[static_cast<int64_t>(i) * ldh + j];
+    // ---- set-up: barriers, TMEM, H_gg and its derived tables
+    if (tid == 0) {
+        mbar_init(&sm.mbar[0], 1);
+        mbar_init(&sm.mbar[1], 1);
+        fence_mbar_init();
+        sm.kappa_bits = __float_as_uint(1.0f);
+        sm.kappa_d_bits = 0u;
+        sm.hmax_bits = 0u;
+        sm.exact_block = 0;
+        sm.abort = 0;
     }
-    if (tid == 0) sm.kappa_bits = __float_as_uint(1.0f);
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, kTcTmemCols);
+        tmem_relinquish();
+        tc_fence_before();
+    }
+    const float* Hg = H + static_cast<int64_t>(g) * kGroup * ldh + static_cast<int64_t>(g) * kGroup;
+    for (int x = tid; x < 32 * 32; x += kTcRows) {
+        const int i = x >> 5, j = x & 31;
+        sm.u.hfull[i][j] = Hg[static_cast<int64_t>(i) * ldh + j];
+    }
+    // zero the B tiles (columns k >= 32 of each row are never written below)
+    for (int x = tid; x < (2 * 32 * 128) / 16; x += kTcRows)
+        reinterpret_cast<uint4*>(sm.bhi)[x] = make_uint4(0u, 0u, 0u, 0u);    // bhi and blo are contiguous
     __syncthreads();
-    float* h32f = reinterpret_cast<float*>(sm.h32);
-    float kap = 0.0f;
-    for (int p = tid; p < kTri; p += kSearchThreads) {
-        const int i = tri_row(p), j = tri_col(p);
-        const float a = sm.hfull[i][j], b = sm.hfull[j][i];
-        if (i == j) {
-            h32f[2 * p] = a;
-            h32f[2 * p + 1] = a;
-            sm.h64[p] = static_cast<double>(a);
-        } else {
-            const float hp = __fadd_rn(a, b);
-            h32f[2 * p] = hp;
-            h32f[2 * p + 1] = hp;
-            sm.h64[p] = static_cast<double>(a) + static_cast<double>(b);
-            const double m = fmax(fabs(static_cast<double>(a)), fabs(static_cast<double>(b)));
-            if (m != 0.0) {
-                const double den = sqrt(fabs(static_cast<double>(sm.hfull[i][i])) *
-                                        fabs(static_cast<double>(sm.hfull[j][j])));
-                const double ratio = den > 0.0 ? m / den : 1e300;
-                kap = fmaxf(kap, ratio > 3.0e38 ? __int_as_float(0x7f800000)
-                                                : __double2float_ru(ratio));
+
+    // 1/sqrt|H_ii| rounded up (for kappa): an upper bound of the true reciprocal
+    if (tid < 32) sm.isd[tid] = __fdiv_ru(1.0f, __fsqrt_rd(fabsf(sm.u.hfull[tid][tid])));
+    __syncthreads();
+
+    // H' for the float64 re-score, kappa, and the largest |(H_ij + H_ji)/2|
+    float kap = 0.0f, hmax = 0.0f;
+    for (int x = tid; x < 32 * 32; x += kTcRows) {
+        const int i = x >> 5, j = x & 31;
+        const float a = sm.u.hfull[i][j], b = sm.u.hfull[j][i];
+        const float hs = up(fabs(0.5 * (static_cast<double>(a) + static_cast<double>(b))));
+        hmax = fmaxf(hmax, (hs <= 3.4028234663852886e38f) ? hs : __int_as_float(0x7f800000));
+        if (j == i) {
+            sm.h64[tri_start(i)] = static_cast<double>(a);
+        } else if (j > i) {
+            sm.h64[tri_start(i) + (j - i)] = static_cast<double>(a) + static_cast<double>(b);
+            const float m = fmaxf(fabsf(a), fabsf(b));
+            if (m != 0.0f) {
+                const float ratio = __fmul_ru(__fmul_ru(m, sm.isd[i]), sm.isd[j]);
+                kap = fmaxf(kap, (ratio <= 3.4028234663852886e38f) ? ratio : __int_as_float(0x7f800000));
             }
         }
     }
-    if (tid < 32) reinterpret_cast<float*>(sm.sqrt_diag)[tid] = __fsqrt_ru(fabsf(sm.hfull[tid][tid]));
     atomicMax(&sm.kappa_bits, __float_as_uint(kap));
+    atomicMax(&sm.hmax_bits, __float_as_uint(hmax));
     __syncthreads();
 
-    const int r = blockIdx.x * kSearchThreads + tid;
-    if (r >= R) return;
-    const float kappa = __uint_as_float(sm.kappa_bits);
-    const float bound_c = kBoundC * kappa;
+    // scale of the block: 2^13 <= hmax * sigma_H < 2^14
+    const float hmx = __uint_as_float(sm.hmax_bits);
+    const bool hbad = !(hmx >= 1.0e-30f) || !(hmx <= 1.0e30f);
+    const int eh = hbad ? 0 : static_cast<int>((__float_as_uint(hmx) >> 23) & 0xFF) - 127;
+    const float sigH = __uint_as_float(static_cast<uint32_t>(127 + 13 - eh) << 23);
+    if (tid < 32) {
+        const float sd = hbad ? 0.0f : __fsqrt_ru(__fmul_ru(fabsf(sm.u.hfull[tid][tid]), sigH));
+        sm.sd[tid] = sd;
+        sm.isd[tid] = __fdiv_ru(1.0f, sd);          // for kappa_d (inf when sd = 0)
+    }
+    __syncthreads();
 
-    float w[32];
-    const float4* wp = reinterpret_cast<const float4*>(W + static_cast<int64_t>(r) * C + g * kGroup);
+    // binary16 split of the scaled symmetrised block; entry (k, n) goes to row n, column k of B
+    float kapd = 0.0f;
+    for (int x = tid; x < 32 * 32; x += kTcRows) {
+        const int k = x >> 5, n = x & 31;
+        const double s = 0.5 * (static_cast<double>(sm.u.hfull[k][n]) + static_cast<double>(sm.u.hfull[n][k])) *
+                         static_cast<double>(sigH);
+        __half hi = __float2half_rn(static_cast<float>(s));
+        if (!(fabsf(__half2float(hi)) >= 6.103515625e-05f)) hi = __float2half_rn(0.0f);   // no subnormal parts
+        const double r1 = s - static_cast<double>(__half2float(hi));
+        __half lo = __float2half_rn(static_cast<float>(r1));
+        if (!(fabsf(__half2float(lo)) >= 6.103515625e-05f)) lo = __float2half_rn(0.0f);
+        const float dlt = up(fabs(r1 - static_cast<double>(__half2float(lo))));
+        if (dlt != 0.0f) {
+            const float ratio = __fmul_ru(__fmul_ru(dlt, sm.isd[k]), sm.isd[n]);
+            kapd = fmaxf(kapd, (ratio <= 3.4028234663852886e38f) ? ratio : __int_as_float(0x7f800000));
+        }
+        const uint32_t off = sw128_off(static_cast<uint32_t>(n), static_cast<uint32_t>(k >> 3)) + (k & 7) * 2;
+        *reinterpret_cast<__half*>(sm.bhi + off) = hi;
+        *reinterpret_cast<__half*>(sm.blo + off) = lo;
+    }
+    atomicMax(&sm.kappa_d_bits, __float_as_uint(kapd));
+    __syncthreads();
+    if (tid == 0) {
+        const double kp = static_cast<double>(__uint_as_float(sm.kappa_bits));
+        const double kd = static_cast<double>(__uint_as_float(sm.kappa_d_bits));
+        double ts = 0.0;
+        for (int i = 0; i < 32; ++i) ts += static_cast<double>(sm.sd[i]);
+        const double tau = 7.62939453125e-06;                         // 2^-17
+        const double c = (kp + kd) * (tau + 1.9073486328125e-06 + 2.384185791015625e-07) + kd +
+                         kp * (9.5367431640625e-07 + 1.1920928955078125e-07);
+        sm.coef = up(c * 1.02);
+        sm.coef_f = up((kp + kd) * 2.44140625e-04 * 1.02);            // 2^-12
+        sm.tsum = up(ts * (1.0 + 1e-6));
+        sm.exact_block = (hbad || !(sm.coef <= 1.0e30f) || !(sm.coef_f <= 1.0e30f)) ? 1 : 0;
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const TcBound tb{sm.coef, sm.coef_f, sm.tsum};
+    const bool exact_block = sm.exact_block != 0;
+
+    // ---- this thread's row
+    const int r = blockIdx.x * kTcRows + tid;
+    const bool valid = r < R;
+    const float* wrow = W + static_cast<int64_t>(valid ? r : 0) * C + g * kGroup;
+    float2 ws[16];
+    if (valid) {
+        const float4* wp = reinterpret_cast<const float4*>(wrow);
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
-        const float4 x = __ldg(wp + v);
-        w[4 * v] = x.x; w[4 * v + 1] = x.y; w[4 * v + 2] = x.z; w[4 * v + 3] = x.w;
+        for (int c = 0; c < 8; ++c) {
+            const float4 x = __ldg(wp + c);
+            ws[2 * c] = make_float2(x.x, x.y);
+            ws[2 * c + 1] = make_float2(x.z, x.w);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) ws[j] = make_float2(0.0f, 0.0f);
     }
     float m = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 32; ++i) m = fmaxf(m, fabsf(w[i]));
-    const int64_t out = static_cast<int64_t>(r) * G + g;
-    if (m == 0.0f) {   // all-zero group: every candidate has zero error
-        delta_out[out] = 0.0f;
-        idx_out[out] = 0;
-        if (err_out) err_out[out] = 0.0f;
-        return;
-    }
+    for (int j = 0; j < 16; ++j) m = fmaxf(m, fmaxf(fabsf(ws[j].x), fabsf(ws[j].y)));
+    const bool zero = (m == 0.0f);
     const float base = __fdiv_rn(m, 7.0f);
-    float* wslot = sm.wslot + tid * kSlot;
-    float* eslot = sm.eslot + tid * kSlot;
-    {
-        float4* w4 = reinterpret_cast<float4*>(wslot);
+    // exact_row: the power-of-two row scale would leave binary32 range; re-score every candidate
+    const bool exact_row = exact_block || !(m >= 7.888609052210118e-31f);      // 2^-100
+    const int em = exact_row ? 0 : static_cast<int>((__float_as_uint(m) >> 23) & 0xFF) - 127;
+    const float sig = __uint_as_float(static_cast<uint32_t>(127 + 13 - em) << 23);
+    const bool screen = valid && !zero && !exact_row;
 #pragma unroll
-        for (int v = 0; v < 8; ++v) w4[v] = make_float4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
-    }
+    for (int j = 0; j < 16; ++j)
+        ws[j] = screen ? make_float2(__fmul_rn(ws[j].x, sig), __fmul_rn(ws[j].y, sig)) : make_float2(0.0f, 0.0f);
+    float* eslot = sm.u.eslot + tid * kTcSlot;
+    const uint32_t swz = static_cast<uint32_t>(tid) & 7u;
+    const uint32_t a0 = smem_u32(sm.a);
+    const uint32_t a_row = a0 + static_cast<uint32_t>(tid) * 128u;
+    const uint32_t bh = smem_u32(sm.bhi), bl = smem_u32(sm.blo);
+    const uint32_t tlane = tmem + (static_cast<uint32_t>(warp * 32) << 16);   // this warp's lanes
+    const bool lane0 = (tid & 31) == 0;
 
     TopK4 top;
     top.init();
     float upper = __int_as_float(0x7f800000);
-    float2 w2[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i) w2[i] = make_float2(w[i], w[i]);
+    bool ok = true;
+
+    // prologue: candidate 0 into stage 0
+    float S0 = tc_quantize(ws, __fmul_rn(__ldg(alpha), base), sig, screen, wrow, eslot, sm.sd, a_row, swz, 0u,
+                           tlane + 32u);
+    float S1 = 0.0f;
+    tmem_st_wait();
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) tc_issue(tmem, a0, bh, bl, &sm.mbar[0]);
+
+    // steady state, two candidates per trip so the stages alternate statically: quantize
+    // candidate k + 1 into the other stage, hand it to the tensor core, then consume k
     for (int k = 0; k < K; k += 2) {
-        const int k1 = (k + 1 < K) ? k + 1 : k;
-        const float2 dk = make_float2(__fmul_rn(__ldg(alpha + k), base), __fmul_rn(__ldg(alpha + k1), base));
-        float2 e[32];
-        group_error_pair(w2, dk, e, wslot, eslot);
-        const float2 E = quad_form_pair<NCH>(sm.h32, e);
-        float S0 = 0.0f, S1 = 0.0f;
-#pragma unroll
-        for (int v = 0; v < 8; ++v) {
-            const float4 s4 = sm.sqrt_diag[v];
-            S0 = fmaf(fabsf(e[4 * v + 0].x), s4.x, S0);
-            S1 = fmaf(fabsf(e[4 * v + 0].y), s4.x, S1);
-            S0 = fmaf(fabsf(e[4 * v + 1].x), s4.y, S0);
-            S1 = fmaf(fabsf(e[4 * v + 1].y), s4.y, S1);
-            S0 = fmaf(fabsf(e[4 * v + 2].x), s4.z, S0);
-            S1 = fmaf(fabsf(e[4 * v + 2].y), s4.z, S1);
-            S0 = fmaf(fabsf(e[4 * v + 3].x), s4.w, S0);
-            S1 = fmaf(fabsf(e[4 * v + 3].y), s4.w, S1);
+        if (k + 1 < K) {
+            S1 = tc_quantize(ws, __fmul_rn(__ldg(alpha + k + 1), base), sig, screen, wrow, eslot, sm.sd, a_row, swz,
+                             1u, tlane + kTcStageCols + 32u);
+            tmem_st_wait();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            if (__syncthreads_or(!ok)) { ok = false; break; }
+            if (lane0 && warp == ((k + 1) & 3)) tc_issue(tmem + kTcStageCols, a0 + 64u, bh, bl, &sm.mbar[1]);
         }
-        const float b0 = bound_c * S0 * S0;
-        upper = fminf(upper, E.x + b0);
-        top.insert(E.x - b0, k);
-        if (k1 != k) {
-            const float b1 = bound_c * S1 * S1;
-            upper = fminf(upper, E.y + b1);
-            top.insert(E.y - b1, k1);
+        if (ok) ok = tc_consume(k, tlane, &sm.mbar[0], &sm.abort, limit_ns, S0, tb, top, upper);
+        if (k + 1 >= K) break;
+        if (k + 2 < K) {
+            S0 = tc_quantize(ws, __fmul_rn(__ldg(alpha + k + 2), base), sig, screen, wrow, eslot, sm.sd, a_row, swz,
+                             0u, tlane + 32u);
+            tmem_st_wait();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            if (__syncthreads_or(!ok)) { ok = false; break; }
+            if (lane0 && warp == ((k + 2) & 3)) tc_issue(tmem, a0, bh, bl, &sm.mbar[0]);
         }
+        if (ok) ok = tc_consume(k + 1, tlane + kTcStageCols, &sm.mbar[1], &sm.abort, limit_ns, S1, tb, top, upper);
     }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, kTcTmemCols);
+    if (!ok) return;
 
     // ---- float64 re-score of every candidate the screening could not exclude
     int nfin = 0;
 #pragma unroll
     for (int a = 0; a < 4; ++a) nfin += (top.k[a] >= 0 && top.L[a] <= upper) ? 1 : 0;
-    const bool overflow = (nfin == 4 && K > 4) || nfin == 0;
+    // a row whose four smallest lower bounds all reach the upper bound is re-scored over every
+    // candidate, by the whole warp (one row at a time, candidates spread over the lanes)
+    const bool overflow = valid && !zero && (!screen || (nfin == 4 && K > 4) || nfin == 0);
+    const int lane = tid & 31;
     double best = 0.0;
     int best_k = -1;
-    const int count = overflow ? K : nfin;
-    for (int a = 0; a < count; ++a) {
-        const int kk = overflow ? a : (a == 0 ? top.k[0] : a == 1 ? top.k[1] : a == 2 ? top.k[2] : top.k[3]);
-        const double E = quad_form64(sm.h64, w, __fmul_rn(__ldg(alpha + kk), base));
-        if (best_k < 0 || E < best || (E == best && kk < best_k)) { best = E; best_k = kk; }
+    unsigned pending = __ballot_sync(0xffffffffu, overflow);
+    while (pending) {
+        const int src = __ffs(pending) - 1;
+        pending &= pending - 1;
+        const float* wsrc = W + static_cast<int64_t>(blockIdx.x * kTcRows + warp * 32 + src) * C + g * kGroup;
+        const float bsrc = __shfl_sync(0xffffffffu, base, src);
+        float wv[32];
+        {
+            const float4* wp = reinterpret_cast<const float4*>(wsrc);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float4 x = __ldg(wp + c);
+                wv[4 * c] = x.x; wv[4 * c + 1] = x.y; wv[4 * c + 2] = x.z; wv[4 * c + 3] = x.w;
+            }
+        }
+        double lb = 0.0;
+        int lk = -1;
+        for (int kk = lane; kk < K; kk += 32) {
+            const double E = tc_quad_form64(sm.h64, wv, __fmul_rn(__ldg(alpha + kk), bsrc));
+            if (lk < 0 || E < lb) { lb = E; lk = kk; }            // kk ascending: ties keep the smaller
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {                          // argmin, smallest k on ties
+            const double ob = __shfl_xor_sync(0xffffffffu, lb, o);
+            const int ok2 = __shfl_xor_sync(0xffffffffu, lk, o);
+            if (ok2 >= 0 && (lk < 0 || ob < lb || (ob == lb && ok2 < lk))) { lb = ob; lk = ok2; }
+        }
+        if (lane == src) { best = lb; best_k = lk; }
+    }
+    if (!valid) return;
+    const int64_t out = static_cast<int64_t>(r) * G + g;
+    if (zero) {   // all-zero group: every candidate has zero error
+        delta_out[out] = 0.0f;
+        idx_out[out] = 0;
+        if (err_out) err_out[out] = 0.0f;
+        return;
+    }
+    if (!overflow) {
+        float wv[32];
+        {
+            const float4* wp = reinterpret_cast<const float4*>(wrow);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float4 x = __ldg(wp + c);
+                wv[4 * c] = x.x; wv[4 * c + 1] = x.y; wv[4 * c + 2] = x.z; wv[4 * c + 3] = x.w;
+            }
+        }
+        for (int a = 0; a < nfin; ++a) {
+            const int kk = a == 0 ? top.k[0] : a == 1 ? top.k[1] : a == 2 ? top.k[2] : top.k[3];
+            const double E = tc_quad_form64(sm.h64, wv, __fmul_rn(__ldg(alpha + kk), base));
+            if (best_k < 0 || E < best || (E == best && kk < best_k)) { best = E; best_k = kk; }
+        }
     }
     delta_out[out] = __fmul_rn(__ldg(alpha + best_k), base);
     idx_out[out] = best_k;
