@@ -53,8 +53,8 @@ CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.a
 # --------------------------------------------------------------------------- setup
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_1b_up_proj.md")
 STAGE_KERNELS = {"hessian": ["hessian_pair_kernel", "hessian_reduce_kernel"],
-                 "scale_search": ["scale_search_kernel"], "lsq_fwd_bwd": ["lsq_kernel"],
-                 "pack_w4a16": ["pack_w4a16_kernel"]}
+                 "scale_search": ["scale_search_kernel"], "lsq_fwd_bwd": ["lsq_blocks_kernel"],
+                 "pack_w4a16": ["pack_w4a16_blocks_kernel"]}
 
 
 STEP_SOURCES = ("device_common.cuh", "hessian.cuh", "lsq_pack.cuh", "scale_search.cuh")

@@ -5,20 +5,16 @@
 // Layout: W, G, Q, grad_W are flat [R*C] arrays; since C % 32 == 0 the group
 // of flat element e is e / 32 and the per-group arrays are flat [R*C/32].
 //
-// Mapping: a warp streams 128 consecutive elements per step; lane l owns the
+// Mapping: a warp streams 128 consecutive elements per load; lane l owns the
 // float4 at elements 4l..4l+3, so 8 lanes cover one group of 32 and the warp
 // covers 4 groups.  Loads and stores are 128-bit and fully coalesced; the
 // per-group step-gradient sum is a 3-level xor butterfly inside each 8-lane
-// segment.  Each warp processes kUnroll steps per loop iteration with all of
-// their loads issued first, to keep enough bytes in flight for HBM3e.
+// segment.
 #pragma once
 
 #include "device_common.cuh"
 
 namespace qat4 {
-
-constexpr int kStreamThreads = 256;
-constexpr int kUnroll = 2;
 
 struct Bf16x4 { uint32_t lo, hi; };
 
@@ -52,59 +48,56 @@ __device__ __forceinline__ LsqElem lsq_elem(float w, float d, float g) {
     return o;
 }
 
-// FWD: write Q.  BWD: write grad_W and grad_delta.  U steps in flight per warp.
-template <typename GT, bool FWD, bool BWD, int U = kUnroll>
-__global__ void __launch_bounds__(kStreamThreads)
-lsq_kernel(const float* __restrict__ W, const float* __restrict__ delta,
-           const GT* __restrict__ G, int64_t nquads, float grad_scale,
-           float* __restrict__ Q, float* __restrict__ grad_W, float* __restrict__ grad_delta) {
+// FWD: write Q.  BWD: write grad_W and grad_delta.  A 128-thread block takes
+// 128 * U consecutive quads (thread t: quads base + u * 128 + t, so 8
+// consecutive lanes hold one group for the butterfly), issues all of its loads,
+// then computes and stores; no thread runs a second iteration.  Blocks are
+// short-lived and plentiful: the block scheduler starts a new one as soon as
+// one finishes, so every SM keeps its loads in flight from the first wave to
+// the last (a grid-stride loop over a fixed grid measured 7% slower: its last
+// round of iterations leaves warps idle).
+constexpr int kLsqBlock = 128;
+template <typename GT, bool FWD, bool BWD, int U>
+__global__ void __launch_bounds__(kLsqBlock)
+lsq_blocks_kernel(const float* __restrict__ W, const float* __restrict__ delta,
+                  const GT* __restrict__ G, int64_t nquads, float grad_scale,
+                  float* __restrict__ Q, float* __restrict__ grad_W, float* __restrict__ grad_delta) {
     const int lane = threadIdx.x & 31;
-    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kStreamThreads + threadIdx.x) >> 5;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kStreamThreads) >> 5;
-    const int64_t nsteps = nquads >> 5;  // nquads is a multiple of 8; handle tail below
-    const int64_t nsteps_ceil = (nquads + 31) >> 5;
-    (void)nsteps;
-
-    for (int64_t s0 = warp * U; s0 < nsteps_ceil; s0 += nwarps * U) {
-        float4 w[U], g[U];
-        float d[U];
-        bool valid[U];
+    const int64_t base = static_cast<int64_t>(blockIdx.x) * (kLsqBlock * U) + threadIdx.x;
+    float4 w[U], g[U];
+    float d[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t quad = (s0 + u) * 32 + lane;
-            valid[u] = quad < nquads;
-            if (valid[u]) {
-                w[u] = __ldcs(reinterpret_cast<const float4*>(W) + quad);
-                d[u] = __ldg(delta + (quad >> 3));
-                if (BWD) g[u] = load_g4<GT>(G, quad);
-            } else {
-                w[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                d[u] = 0.f;
-                g[u] = w[u];
-            }
+    for (int u = 0; u < U; ++u) {
+        const int64_t quad = base + u * kLsqBlock;
+        if (quad < nquads) {
+            w[u] = __ldcs(reinterpret_cast<const float4*>(W) + quad);
+            d[u] = __ldg(delta + (quad >> 3));
+            if (BWD) g[u] = load_g4<GT>(G, quad);
+        } else {
+            w[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            d[u] = 0.f;
+            g[u] = w[u];
         }
+    }
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t quad = (s0 + u) * 32 + lane;
-            const LsqElem e0 = lsq_elem(w[u].x, d[u], BWD ? g[u].x : 0.f);
-            const LsqElem e1 = lsq_elem(w[u].y, d[u], BWD ? g[u].y : 0.f);
-            const LsqElem e2 = lsq_elem(w[u].z, d[u], BWD ? g[u].z : 0.f);
-            const LsqElem e3 = lsq_elem(w[u].w, d[u], BWD ? g[u].w : 0.f);
-            if (FWD && valid[u])
-                __stcs(reinterpret_cast<float4*>(Q) + quad, make_float4(e0.q, e1.q, e2.q, e3.q));
-            if (BWD) {
-                if (valid[u])
-                    __stcs(reinterpret_cast<float4*>(grad_W) + quad,
-                           make_float4(e0.gw, e1.gw, e2.gw, e3.gw));
-                float acc = g[u].x * e0.dq;
-                acc = fmaf(g[u].y, e1.dq, acc);
-                acc = fmaf(g[u].z, e2.dq, acc);
-                acc = fmaf(g[u].w, e3.dq, acc);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-                if (valid[u] && (lane & 7) == 0) grad_delta[quad >> 3] = grad_scale * acc;
-            }
+    for (int u = 0; u < U; ++u) {
+        const int64_t quad = base + u * kLsqBlock;
+        const bool valid = quad < nquads;
+        const LsqElem e0 = lsq_elem(w[u].x, d[u], BWD ? g[u].x : 0.f);
+        const LsqElem e1 = lsq_elem(w[u].y, d[u], BWD ? g[u].y : 0.f);
+        const LsqElem e2 = lsq_elem(w[u].z, d[u], BWD ? g[u].z : 0.f);
+        const LsqElem e3 = lsq_elem(w[u].w, d[u], BWD ? g[u].w : 0.f);
+        if (FWD && valid) __stcs(reinterpret_cast<float4*>(Q) + quad, make_float4(e0.q, e1.q, e2.q, e3.q));
+        if (BWD) {
+            if (valid) __stcs(reinterpret_cast<float4*>(grad_W) + quad, make_float4(e0.gw, e1.gw, e2.gw, e3.gw));
+            float acc = g[u].x * e0.dq;
+            acc = fmaf(g[u].y, e1.dq, acc);
+            acc = fmaf(g[u].z, e2.dq, acc);
+            acc = fmaf(g[u].w, e3.dq, acc);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            if (valid && (lane & 7) == 0) grad_delta[quad >> 3] = grad_scale * acc;
         }
     }
 }
@@ -155,40 +148,35 @@ __device__ __forceinline__ uint32_t pack8(float4 a, float4 b, float d) {
     return out;
 }
 
-// W4A16 export.  A warp step covers 256 consecutive weights; lane l converts
-// weights 8l..8l+7 (one group is four lanes, so one reciprocal per lane) into
-// one 32-bit word, and the warp stores 128 contiguous bytes.  Lanes 0, 4, ...,
-// 28 also write their group's binary16 scale.  U steps in flight per warp.
-template <int U = 2, int NT = kStreamThreads>
-__global__ void __launch_bounds__(NT)
-pack_w4a16_kernel(const float* __restrict__ W, const float* __restrict__ delta, int64_t noct,
-                  uint32_t* __restrict__ packed32, uint16_t* __restrict__ scales) {
-    const int lane = threadIdx.x & 31;
-    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * NT + threadIdx.x) >> 5;
-    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * NT) >> 5;
-    const int64_t nsteps_ceil = (noct + 31) >> 5;    // noct = number of 8-weight octets
-    for (int64_t s0 = warp * U; s0 < nsteps_ceil; s0 += nwarps * U) {
-        float4 wa[U], wb[U];
-        float d[U];
+// W4A16 export as many short blocks: a 128-thread block converts 128 * U
+// consecutive octets (thread t: octets base + u * 128 + t, u < U, so each warp
+// load covers 1 KB contiguous), issuing all of its loads before converting any.
+// Blocks are short-lived and plentiful; the block scheduler starts a new one as
+// soon as one finishes, so the loads in flight per SM stay high from the first
+// wave to the last and no thread runs a second iteration.
+constexpr int kPackBlock = 128;
+template <int U>
+__global__ void __launch_bounds__(kPackBlock)
+pack_w4a16_blocks_kernel(const float* __restrict__ W, const float* __restrict__ delta, int64_t noct,
+                         uint32_t* __restrict__ packed32, uint16_t* __restrict__ scales) {
+    const int64_t base = static_cast<int64_t>(blockIdx.x) * (kPackBlock * U) + threadIdx.x;
+    float4 a[U], b[U];
+    float d[U];
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t oct = (s0 + u) * 32 + lane;
-            if (oct < noct) {
-                wa[u] = __ldcs(reinterpret_cast<const float4*>(W) + 2 * oct);
-                wb[u] = __ldcs(reinterpret_cast<const float4*>(W) + 2 * oct + 1);
-                d[u] = __ldg(delta + (oct >> 2));
-            } else {
-                wa[u] = wb[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                d[u] = 0.f;
-            }
+    for (int u = 0; u < U; ++u) {
+        const int64_t o = base + u * kPackBlock;
+        if (o < noct) {
+            a[u] = __ldcs(reinterpret_cast<const float4*>(W) + 2 * o);
+            b[u] = __ldcs(reinterpret_cast<const float4*>(W) + 2 * o + 1);
+            d[u] = __ldg(delta + (o >> 2));
         }
+    }
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int64_t oct = (s0 + u) * 32 + lane;
-            if (oct < noct) {
-                __stcs(packed32 + oct, pack8(wa[u], wb[u], d[u]));
-                if ((lane & 3) == 0) scales[oct >> 2] = __half_as_ushort(__float2half_rn(d[u]));
-            }
+    for (int u = 0; u < U; ++u) {
+        const int64_t o = base + u * kPackBlock;
+        if (o < noct) {
+            __stcs(packed32 + o, pack8(a[u], b[u], d[u]));
+            if ((o & 3) == 0) scales[o >> 2] = __half_as_ushort(__float2half_rn(d[u]));
         }
     }
 }

@@ -66,16 +66,6 @@ qat4_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? QAT4_OK : QAT4_ERR_CUDA;
 }
 
-// Blocks for a grid-stride streaming kernel over `nquads` float4 quads:
-// enough warps to cover the work once, at most 8 resident blocks per SM.
-unsigned stream_blocks(int64_t nquads, int sms, int unroll) {
-    const int64_t warp_steps = (nquads + 31) / 32;
-    const int64_t warps_needed = (warp_steps + unroll - 1) / unroll;
-    const int64_t blocks_needed = (warps_needed + (qat4::kStreamThreads / 32) - 1) / (qat4::kStreamThreads / 32);
-    const int64_t cap = static_cast<int64_t>(sms) * (2048 / qat4::kStreamThreads);
-    return static_cast<unsigned>(std::max<int64_t>(1, std::min(blocks_needed, cap)));
-}
-
 // --------------------------------------------------------------- tensor maps
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -237,28 +227,34 @@ static qat4_status lsq_common(const float* W, const float* delta, const void* G,
     int dev;
     DeviceInfo* info;
     if (!device_info(&dev, &info)) return QAT4_ERR_CUDA;
+    // short 128-thread blocks, two quads per thread, all loads issued up front; R * C <= 2^40
+    // keeps the grid below 2^32 blocks
     const int64_t nquads = R * C / 4;
-    const unsigned blocks = stream_blocks(nquads, info->sms, qat4::kUnroll);
-    const unsigned th = qat4::kStreamThreads;
+    constexpr int kU = 2;
+    const unsigned blocks = static_cast<unsigned>((nquads + qat4::kLsqBlock * kU - 1) / (qat4::kLsqBlock * kU));
+    const unsigned th = qat4::kLsqBlock;
     if (fwd && !bwd) {
-        qat4::lsq_kernel<float, true, false><<<blocks, th, 0, stream>>>(W, delta, nullptr, nquads, 0.f, Q,
-                                                                       nullptr, nullptr);
+        qat4::lsq_blocks_kernel<float, true, false, kU><<<blocks, th, 0, stream>>>(W, delta, nullptr, nquads, 0.f, Q,
+                                                                                  nullptr, nullptr);
     } else if (g_dtype == QAT4_F32) {
         const float* g = static_cast<const float*>(G);
         if (fwd)
-            qat4::lsq_kernel<float, true, true><<<blocks, th, 0, stream>>>(W, delta, g, nquads, grad_scale, Q,
-                                                                          grad_W, grad_delta);
+            qat4::lsq_blocks_kernel<float, true, true, kU><<<blocks, th, 0, stream>>>(W, delta, g, nquads, grad_scale,
+                                                                                     Q, grad_W, grad_delta);
         else
-            qat4::lsq_kernel<float, false, true><<<blocks, th, 0, stream>>>(W, delta, g, nquads, grad_scale,
-                                                                           nullptr, grad_W, grad_delta);
+            qat4::lsq_blocks_kernel<float, false, true, kU><<<blocks, th, 0, stream>>>(W, delta, g, nquads,
+                                                                                      grad_scale, nullptr, grad_W,
+                                                                                      grad_delta);
     } else {
         const uint16_t* g = static_cast<const uint16_t*>(G);
         if (fwd)
-            qat4::lsq_kernel<uint16_t, true, true><<<blocks, th, 0, stream>>>(W, delta, g, nquads, grad_scale,
-                                                                             Q, grad_W, grad_delta);
+            qat4::lsq_blocks_kernel<uint16_t, true, true, kU><<<blocks, th, 0, stream>>>(W, delta, g, nquads,
+                                                                                        grad_scale, Q, grad_W,
+                                                                                        grad_delta);
         else
-            qat4::lsq_kernel<uint16_t, false, true><<<blocks, th, 0, stream>>>(W, delta, g, nquads, grad_scale,
-                                                                              nullptr, grad_W, grad_delta);
+            qat4::lsq_blocks_kernel<uint16_t, false, true, kU><<<blocks, th, 0, stream>>>(W, delta, g, nquads,
+                                                                                         grad_scale, nullptr, grad_W,
+                                                                                         grad_delta);
     }
     return launch_status();
 }
@@ -290,8 +286,11 @@ qat4_status qat4_pack_w4a16(const float* W, const float* delta, int64_t R, int64
     int dev;
     DeviceInfo* info;
     if (!device_info(&dev, &info)) return QAT4_ERR_CUDA;
+    // 128-thread blocks of 4 octets per thread; R * C <= 2^40 keeps the grid below 2^28 blocks
     const int64_t noct = R * C / 8;   // C % 32 == 0: octets never straddle a group
-    qat4::pack_w4a16_kernel<2><<<stream_blocks(noct, info->sms, 2), qat4::kStreamThreads, 0, stream>>>(
+    constexpr int kU = 4;
+    const int64_t blocks = (noct + qat4::kPackBlock * kU - 1) / (qat4::kPackBlock * kU);
+    qat4::pack_w4a16_blocks_kernel<kU><<<static_cast<unsigned>(blocks), qat4::kPackBlock, 0, stream>>>(
         W, delta, noct, reinterpret_cast<uint32_t*>(packed), scales);
     return launch_status();
 }
