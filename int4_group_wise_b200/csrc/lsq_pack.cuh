@@ -154,21 +154,37 @@ __device__ __forceinline__ uint32_t pack8(float4 a, float4 b, float d) {
 // Blocks are short-lived and plentiful; the block scheduler starts a new one as
 // soon as one finishes, so the loads in flight per SM stay high from the first
 // wave to the last and no thread runs a second iteration.
+//
+// ROW selects the per-channel export (one scale per row of `row_oct` octets):
+// the row of an octet is found by a binary64 multiply with 1/row_oct and a
+// one-step correction (exact for any octet index below 2^52), and the first
+// octet of a row writes the row's scale.  Otherwise the scale index is the
+// group, octet / 4.
 constexpr int kPackBlock = 128;
-template <int U>
+template <int U, bool ROW>
 __global__ void __launch_bounds__(kPackBlock)
 pack_w4a16_blocks_kernel(const float* __restrict__ W, const float* __restrict__ delta, int64_t noct,
+                         int64_t row_oct, double inv_row_oct,
                          uint32_t* __restrict__ packed32, uint16_t* __restrict__ scales) {
     const int64_t base = static_cast<int64_t>(blockIdx.x) * (kPackBlock * U) + threadIdx.x;
     float4 a[U], b[U];
     float d[U];
+    int64_t si[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
         const int64_t o = base + u * kPackBlock;
+        if (ROW) {
+            int64_t r = __double2ll_rz(__ll2double_rn(o) * inv_row_oct);
+            if (r * row_oct > o) --r;
+            else if ((r + 1) * row_oct <= o) ++r;
+            si[u] = r;
+        } else {
+            si[u] = o >> 2;
+        }
         if (o < noct) {
             a[u] = __ldcs(reinterpret_cast<const float4*>(W) + 2 * o);
             b[u] = __ldcs(reinterpret_cast<const float4*>(W) + 2 * o + 1);
-            d[u] = __ldg(delta + (o >> 2));
+            d[u] = __ldg(delta + si[u]);
         }
     }
 #pragma unroll
@@ -176,7 +192,8 @@ pack_w4a16_blocks_kernel(const float* __restrict__ W, const float* __restrict__ 
         const int64_t o = base + u * kPackBlock;
         if (o < noct) {
             __stcs(packed32 + o, pack8(a[u], b[u], d[u]));
-            if ((o & 3) == 0) scales[o >> 2] = __half_as_ushort(__float2half_rn(d[u]));
+            const bool first = ROW ? (o == si[u] * row_oct) : ((o & 3) == 0);
+            if (first) scales[si[u]] = __half_as_ushort(__float2half_rn(d[u]));
         }
     }
 }

@@ -290,8 +290,8 @@ qat4_status qat4_pack_w4a16(const float* W, const float* delta, int64_t R, int64
     const int64_t noct = R * C / 8;   // C % 32 == 0: octets never straddle a group
     constexpr int kU = 4;
     const int64_t blocks = (noct + qat4::kPackBlock * kU - 1) / (qat4::kPackBlock * kU);
-    qat4::pack_w4a16_blocks_kernel<kU><<<static_cast<unsigned>(blocks), qat4::kPackBlock, 0, stream>>>(
-        W, delta, noct, reinterpret_cast<uint32_t*>(packed), scales);
+    qat4::pack_w4a16_blocks_kernel<kU, false><<<static_cast<unsigned>(blocks), qat4::kPackBlock, 0, stream>>>(
+        W, delta, noct, 4, 0.25, reinterpret_cast<uint32_t*>(packed), scales);
     return launch_status();
 }
 
@@ -354,8 +354,13 @@ qat4_status qat4_pack_w4a16_rowwise(const float* W, const float* delta, int64_t 
     if (!W || !delta || !packed || !scales) return QAT4_ERR_NULL;
     if (!valid_rc(R, C)) return QAT4_ERR_SHAPE;
     if (!aligned16(W) || !aligned16(delta) || !aligned16(packed) || !aligned16(scales)) return QAT4_ERR_ALIGN;
-    qat4::pack_w4a16_rowwise_kernel<<<static_cast<unsigned>(R), qat4::kRowThreads, 0, stream>>>(
-        W, delta, static_cast<int>(C), reinterpret_cast<uint32_t*>(packed), scales);
+    // the short-block export in its row mode: C / 8 octets share one scale
+    const int64_t noct = R * C / 8;
+    constexpr int kU = 4;
+    const int64_t blocks = (noct + qat4::kPackBlock * kU - 1) / (qat4::kPackBlock * kU);
+    const int64_t row_oct = C / 8;
+    qat4::pack_w4a16_blocks_kernel<kU, true><<<static_cast<unsigned>(blocks), qat4::kPackBlock, 0, stream>>>(
+        W, delta, noct, row_oct, 1.0 / static_cast<double>(row_oct), reinterpret_cast<uint32_t*>(packed), scales);
     return launch_status();
 }
 

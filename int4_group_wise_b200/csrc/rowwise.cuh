@@ -5,9 +5,9 @@
 // weights and is normalised by the caller's grad_scale (1/sqrt(C * 7)).
 //
 // Mapping: one CTA of 256 threads per row.  The row streams through as float4
-// (LSQ) or 8-weight octets (pack) with 128-bit coalesced accesses; the row's
-// step-gradient sum is a warp-shuffle tree followed by a shared-memory sum
-// over the 8 warps.
+// with 128-bit coalesced accesses; the row's step-gradient sum is a
+// warp-shuffle tree followed by a shared-memory sum over the 8 warps.  The
+// per-channel export is the short-block pack of lsq_pack.cuh in its row mode.
 #pragma once
 
 #include "device_common.cuh"
@@ -58,22 +58,6 @@ lsq_rowwise_kernel(const float* __restrict__ W, const float* __restrict__ delta,
             grad_delta[r] = grad_scale * s;
         }
     }
-}
-
-__global__ void __launch_bounds__(kRowThreads)
-pack_w4a16_rowwise_kernel(const float* __restrict__ W, const float* __restrict__ delta, int C,
-                          uint32_t* __restrict__ packed32, uint16_t* __restrict__ scales) {
-    const int64_t r = blockIdx.x;
-    const float d = __ldg(delta + r);
-    const int noct = C >> 3;
-    const int64_t o0 = r * noct;
-    for (int i = threadIdx.x; i < noct; i += kRowThreads) {
-        const int64_t oct = o0 + i;
-        const float4 a = __ldcs(reinterpret_cast<const float4*>(W) + 2 * oct);
-        const float4 b = __ldcs(reinterpret_cast<const float4*>(W) + 2 * oct + 1);
-        __stcs(packed32 + oct, pack8(a, b, d));
-    }
-    if (threadIdx.x == 0) scales[r] = __half_as_ushort(__float2half_rn(d));
 }
 
 }  // namespace qat4

@@ -130,3 +130,28 @@ def test_search_full_size_sampled_rows(cfg, cache, oracle_mod):
     H = _diag_block_hessian(cache, cfg, oracle_mod)
     rows = np.arange(0, W.shape[0], 32)
     check_search(W, H, wl.alpha(), oracle_mod, rows=rows)
+
+
+def test_search_degenerate_blocks_rows_and_ties(oracle_mod):
+    """Paths the tensor-core screen hands to the float64 re-score: a 32x32 block of H that is
+    all zero (every candidate ties, so every row is re-scored over all K by its warp), rows whose
+    weights are too small for the power-of-two row scale (|w| < 2^-100), and a grid with repeated
+    multipliers (equal objectives: the smallest index wins)."""
+    rng = np.random.default_rng(12)
+    R, C = 200, 96
+    W = (rng.standard_normal((R, C)) * 0.02).astype(f32)
+    W[5, :] = (rng.standard_normal(C) * 1e-33).astype(f32)          # m ~ 2^-108
+    W[77, 64:96] = (rng.standard_normal(32) * 1e-36).astype(f32)     # one tiny group, H_gg nonzero
+    Xb = inputs.activations(256, C, seed=12, cfg=52, name="X", outliers=2)
+    H = oracle_mod.hessian(Xb).astype(f32)
+    H[32:64, 32:64] = 0.0                                            # group 1: H_gg = 0
+    alpha = inputs.alpha_grid(0.5, 0.01, 51)
+    check_search(W, H, alpha, oracle_mod)
+    d, i, e = q4.scale_search(_dev(W), _dev(H), _dev(alpha))
+    torch.cuda.synchronize()
+    assert torch.all(i[:, 1] == 0) and torch.all(e[:, 1] == 0)       # zero block: all tie at k = 0
+    rep = np.repeat(inputs.alpha_grid(0.6, 0.05, 9), 3).astype(f32)  # each multiplier three times
+    _, i2, _ = q4.scale_search(_dev(W), _dev(H), _dev(rep))
+    torch.cuda.synchronize()
+    assert torch.all(i2 % 3 == 0)                                     # first of each equal triple
+    check_search(W, H, rep, oracle_mod)
