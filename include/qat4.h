@@ -162,6 +162,32 @@ qat4_status qat4_lsq_fwd_bwd(const float *W, const float *delta, const void *G, 
                              int64_t R, int64_t C, float grad_scale,
                              float *Q, float *grad_W, float *grad_delta, cudaStream_t stream);
 
+/* LSQ step of a whole layer from and to HOST memory (the blog's QAT step on
+ * weights that live on the host): the rows are streamed through the GPU in
+ * chunks of about 2 M weights, each chunk uploaded on `stream`, run through
+ * the fused forward/backward kernel, and downloaded on `copy_stream`, so the
+ * uploads of one chunk overlap the downloads of the previous one (PCIe is
+ * full duplex).  Results are identical to qat4_lsq_fwd_bwd on the same data.
+ *
+ *  W, delta, G, Q, grad_W, grad_delta   HOST pointers with the shapes and
+ *            dtypes of qat4_lsq_fwd_bwd; page-locked memory is needed for the
+ *            copies to overlap (pageable memory is correct but serialises).
+ *  workspace DEVICE memory, 256-byte aligned, at least
+ *            qat4_lsq_fwd_bwd_host_workspace_bytes(R, C, g_dtype) bytes
+ *            (two chunks of every operand).
+ *  stream, copy_stream   the call returns once everything is enqueued; when
+ *            `stream` has completed (cudaStreamSynchronize), the outputs are
+ *            on the host.  copy_stream may equal stream (then nothing overlaps).
+ *  The call creates and releases five CUDA events per call; it allocates no
+ *  memory.  Errors: QAT4_ERR_NULL, _SHAPE, _DTYPE, _WORKSPACE, _ALIGN, _CUDA.
+ */
+size_t qat4_lsq_fwd_bwd_host_workspace_bytes(int64_t R, int64_t C, qat4_dtype g_dtype);
+qat4_status qat4_lsq_fwd_bwd_host(const float *W, const float *delta, const void *G, qat4_dtype g_dtype,
+                                  int64_t R, int64_t C, float grad_scale,
+                                  float *Q, float *grad_W, float *grad_delta,
+                                  void *workspace, size_t workspace_bytes,
+                                  cudaStream_t stream, cudaStream_t copy_stream);
+
 /* W4A16 export (model card, "QAT Highlights": the same INT4 grid at
  * initialisation, QAT and export).  Codes are the forward codes
  * clamp(rint(w / Delta), -8, 7) for the float32 Delta.

@@ -8,7 +8,7 @@ device pointers plus the current CUDA stream to the C ABI in
 
 Functions (same names as the C entry points, without the ``qat4_`` prefix):
 ``hessian``, ``hessian_workspace_bytes``, ``hessian_noalloc``, ``scale_search``, ``lsq_fwd``,
-``lsq_bwd``, ``lsq_fwd_bwd``, ``pack_w4a16``, ``sync_check``,
+``lsq_bwd``, ``lsq_fwd_bwd``, ``lsq_fwd_bwd_host``, ``pack_w4a16``, ``sync_check``,
 ``status_string``, ``selftest_bounded_wait``.
 """
 from __future__ import annotations
@@ -40,6 +40,8 @@ EXPORTS = {
     "qat4_lsq_fwd": (ct.c_int, [_P, _P, _I64, _I64, _P, _P]),
     "qat4_lsq_bwd": (ct.c_int, [_P, _P, _P, ct.c_int, _I64, _I64, _F, _P, _P, _P]),
     "qat4_lsq_fwd_bwd": (ct.c_int, [_P, _P, _P, ct.c_int, _I64, _I64, _F, _P, _P, _P, _P]),
+    "qat4_lsq_fwd_bwd_host_workspace_bytes": (_Z, [_I64, _I64, ct.c_int]),
+    "qat4_lsq_fwd_bwd_host": (ct.c_int, [_P, _P, _P, ct.c_int, _I64, _I64, _F, _P, _P, _P, _P, _Z, _P, _P]),
     "qat4_pack_w4a16": (ct.c_int, [_P, _P, _I64, _I64, _P, _P, _P]),
     "qat4_lsq_fwd_rowwise": (ct.c_int, [_P, _P, _I64, _I64, _P, _P]),
     "qat4_lsq_bwd_rowwise": (ct.c_int, [_P, _P, _P, ct.c_int, _I64, _I64, _F, _P, _P, _P]),
@@ -242,6 +244,64 @@ def lsq_fwd_bwd(W, delta, G, grad_scale=GRAD_SCALE, Q=None, grad_W=None, grad_de
                               ct.c_float(grad_scale), _dev(Q, "Q"), _dev(grad_W, "grad_W"),
                               _dev(grad_delta, "grad_delta"), _stream(stream)), "qat4_lsq_fwd_bwd")
     return Q, grad_W, grad_delta
+
+
+def _host(t, name, dtype=None, shape=None):
+    import torch
+    if not isinstance(t, torch.Tensor) or t.is_cuda:
+        raise TypeError(f"{name} must be a host (CPU) tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return ct.c_void_p(t.data_ptr())
+
+
+def lsq_fwd_bwd_host_workspace_bytes(R: int, C: int, g_dtype: int) -> int:
+    return int(lib().qat4_lsq_fwd_bwd_host_workspace_bytes(int(R), int(C), int(g_dtype)))
+
+
+def lsq_fwd_bwd_host(W, delta, G, grad_scale=GRAD_SCALE, Q=None, grad_W=None, grad_delta=None,
+                     workspace=None, stream=None, copy_stream=None):
+    """The fused LSQ step on host tensors (page-locked for overlap), streamed through the current
+    GPU in row chunks; returns host (Q, grad_W, grad_delta).  Asynchronous: synchronize `stream`
+    (default: the current stream) before reading the outputs."""
+    import torch
+    L = lib()
+    _host(W, "W", torch.float32)
+    R, C = W.shape
+    _host(delta, "delta", torch.float32, (R, C // 32))
+    _host(G, "G", None, (R, C))
+    gd = _gdtype(G)
+    pin = W.is_pinned()
+    Q = torch.empty((R, C), dtype=torch.float32, pin_memory=pin) if Q is None else Q
+    grad_W = torch.empty((R, C), dtype=torch.float32, pin_memory=pin) if grad_W is None else grad_W
+    grad_delta = torch.empty((R, C // 32), dtype=torch.float32, pin_memory=pin) if grad_delta is None else grad_delta
+    need = lsq_fwd_bwd_host_workspace_bytes(R, C, gd)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=torch.cuda.current_device())
+    cs = copy_stream if copy_stream is not None else _copy_stream()
+    _check(L.qat4_lsq_fwd_bwd_host(_host(W, "W"), _host(delta, "delta"), _host(G, "G"), gd, R, C,
+                                   ct.c_float(grad_scale), _host(Q, "Q", torch.float32, (R, C)),
+                                   _host(grad_W, "grad_W", torch.float32, (R, C)),
+                                   _host(grad_delta, "grad_delta", torch.float32, (R, C // 32)),
+                                   _dev(workspace, "workspace"), workspace.numel(), _stream(stream),
+                                   ct.c_void_p(cs.cuda_stream)), "qat4_lsq_fwd_bwd_host")
+    return Q, grad_W, grad_delta
+
+
+_copy_streams = {}
+
+
+def _copy_stream():
+    """One side stream per device for the downloads of lsq_fwd_bwd_host."""
+    import torch
+    d = torch.cuda.current_device()
+    if d not in _copy_streams:
+        _copy_streams[d] = torch.cuda.Stream(device=d)
+    return _copy_streams[d]
 
 
 def pack_w4a16(W, delta, packed=None, scales=None, stream=None):

@@ -295,6 +295,97 @@ qat4_status qat4_pack_w4a16(const float* W, const float* delta, int64_t R, int64
     return launch_status();
 }
 
+// ------------------------------------------------- LSQ step from host memory
+// Rows per chunk of the host-buffer pipeline: about 2 M weights, at least one row.
+static int64_t host_chunk_rows(int64_t R, int64_t C) {
+    return std::max<int64_t>(1, std::min<int64_t>(R, (int64_t(1) << 21) / C));
+}
+static size_t host_chunk_bytes(int64_t rows, int64_t C, qat4_dtype g_dtype) {
+    const int64_t n = rows * C;
+    const size_t gb = g_dtype == QAT4_BF16 ? 2 : 4;
+    // W, G, Q, grad_W, delta, grad_delta of one chunk, each rounded up to 256 bytes
+    auto r256 = [](size_t b) { return (b + 255) & ~size_t(255); };
+    return r256(n * 4) + r256(n * gb) + r256(n * 4) + r256(n * 4) + 2 * r256(n / 32 * 4);
+}
+
+size_t qat4_lsq_fwd_bwd_host_workspace_bytes(int64_t R, int64_t C, qat4_dtype g_dtype) {
+    if (!valid_rc(R, C) || (g_dtype != QAT4_F32 && g_dtype != QAT4_BF16)) return 0;
+    return 2 * host_chunk_bytes(host_chunk_rows(R, C), C, g_dtype);
+}
+
+qat4_status qat4_lsq_fwd_bwd_host(const float* W, const float* delta, const void* G, qat4_dtype g_dtype,
+                                  int64_t R, int64_t C, float grad_scale, float* Q, float* grad_W,
+                                  float* grad_delta, void* workspace, size_t workspace_bytes,
+                                  cudaStream_t stream, cudaStream_t copy_stream) {
+    if (!W || !delta || !G || !Q || !grad_W || !grad_delta || !workspace) return QAT4_ERR_NULL;
+    if (!valid_rc(R, C)) return QAT4_ERR_SHAPE;
+    if (g_dtype != QAT4_F32 && g_dtype != QAT4_BF16) return QAT4_ERR_DTYPE;
+    if (workspace_bytes < qat4_lsq_fwd_bwd_host_workspace_bytes(R, C, g_dtype)) return QAT4_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return QAT4_ERR_ALIGN;
+    const int64_t crow = host_chunk_rows(R, C);
+    const size_t gb = g_dtype == QAT4_BF16 ? 2 : 4;
+    const size_t stage = host_chunk_bytes(crow, C, g_dtype);
+    auto r256 = [](size_t b) { return (b + 255) & ~size_t(255); };
+    struct Buf { float *w, *q, *gw, *d, *gd; void* g; };
+    Buf buf[2];
+    for (int b = 0; b < 2; ++b) {
+        uint8_t* p = static_cast<uint8_t*>(workspace) + b * stage;
+        const int64_t n = crow * C;
+        buf[b].w = reinterpret_cast<float*>(p);            p += r256(n * 4);
+        buf[b].g = p;                                       p += r256(n * gb);
+        buf[b].q = reinterpret_cast<float*>(p);            p += r256(n * 4);
+        buf[b].gw = reinterpret_cast<float*>(p);           p += r256(n * 4);
+        buf[b].d = reinterpret_cast<float*>(p);            p += r256(n / 32 * 4);
+        buf[b].gd = reinterpret_cast<float*>(p);
+    }
+    cudaEvent_t done[2], freed[2], last;
+    bool made = true;
+    for (int b = 0; b < 2; ++b) {
+        made &= cudaEventCreateWithFlags(&done[b], cudaEventDisableTiming) == cudaSuccess;
+        made &= cudaEventCreateWithFlags(&freed[b], cudaEventDisableTiming) == cudaSuccess;
+    }
+    made &= cudaEventCreateWithFlags(&last, cudaEventDisableTiming) == cudaSuccess;
+    qat4_status st = made ? QAT4_OK : QAT4_ERR_CUDA;
+    const auto H2D = cudaMemcpyHostToDevice;
+    const auto D2H = cudaMemcpyDeviceToHost;
+    int64_t chunk = 0;
+    for (int64_t r0 = 0; st == QAT4_OK && r0 < R; r0 += crow, ++chunk) {
+        const int b = static_cast<int>(chunk & 1);
+        const int64_t nr = std::min(crow, R - r0);
+        const size_t n = static_cast<size_t>(nr * C);
+        const size_t off = static_cast<size_t>(r0 * C);
+        bool ok = true;
+        // the stage's outputs of two chunks ago must be on the host before it is refilled
+        if (chunk >= 2) ok &= cudaStreamWaitEvent(stream, freed[b], 0) == cudaSuccess;
+        ok &= cudaMemcpyAsync(buf[b].w, W + off, n * 4, H2D, stream) == cudaSuccess;
+        ok &= cudaMemcpyAsync(buf[b].g, static_cast<const uint8_t*>(G) + off * gb, n * gb, H2D, stream) == cudaSuccess;
+        ok &= cudaMemcpyAsync(buf[b].d, delta + off / 32, n / 32 * 4, H2D, stream) == cudaSuccess;
+        if (!ok) { st = QAT4_ERR_CUDA; break; }
+        st = lsq_common(buf[b].w, buf[b].d, buf[b].g, g_dtype, nr, C, grad_scale, buf[b].q, buf[b].gw, buf[b].gd,
+                        true, true, stream);
+        if (st != QAT4_OK) break;
+        ok &= cudaEventRecord(done[b], stream) == cudaSuccess;
+        // downloads on the copy stream overlap the next chunk's uploads (PCIe is full duplex)
+        ok &= cudaStreamWaitEvent(copy_stream, done[b], 0) == cudaSuccess;
+        ok &= cudaMemcpyAsync(Q + off, buf[b].q, n * 4, D2H, copy_stream) == cudaSuccess;
+        ok &= cudaMemcpyAsync(grad_W + off, buf[b].gw, n * 4, D2H, copy_stream) == cudaSuccess;
+        ok &= cudaMemcpyAsync(grad_delta + off / 32, buf[b].gd, n / 32 * 4, D2H, copy_stream) == cudaSuccess;
+        ok &= cudaEventRecord(freed[b], copy_stream) == cudaSuccess;
+        if (!ok) st = QAT4_ERR_CUDA;
+    }
+    // completion is observable on `stream`: it waits for the last download
+    if (made) {
+        if (cudaEventRecord(last, copy_stream) != cudaSuccess || cudaStreamWaitEvent(stream, last, 0) != cudaSuccess)
+            st = QAT4_ERR_CUDA;
+        for (int b = 0; b < 2; ++b) {
+            cudaEventDestroy(done[b]);
+            cudaEventDestroy(freed[b]);
+        }
+        cudaEventDestroy(last);
+    }
+    return st;
+}
+
 // -------------------------------------------------------------- per-channel
 static qat4_status lsq_rowwise_common(const float* W, const float* delta, const void* G, qat4_dtype g_dtype,
                                       int64_t R, int64_t C, float grad_scale, float* Q, float* grad_W,

@@ -128,3 +128,18 @@ def test_refine_validation():
     assert L.qat4_refine(A, 4, 64, A, 66, A, 5, 1, A, A, None, A, 1 << 20, None) == 3      # ldh % 4
     assert L.qat4_refine(A, 4, 64, A, 64, A, 5, 1, A, A, None, A, 16, None) == 5           # workspace
     assert L.qat4_refine_workspace_bytes(4, 64) == 2 * 4 * 64 * 8
+
+
+def test_lsq_host_validation():
+    L = q4.lib()
+    ws = q4.lsq_fwd_bwd_host_workspace_bytes(3000, 1024, q4.QAT4_BF16)
+    assert ws > 0 and q4.lsq_fwd_bwd_host_workspace_bytes(3000, 48, q4.QAT4_BF16) == 0
+    assert q4.lsq_fwd_bwd_host_workspace_bytes(3000, 1024, 7) == 0
+    f = L.qat4_lsq_fwd_bwd_host
+    s = ct.c_float(q4.GRAD_SCALE)
+    assert f(None, A, A, 1, 3000, 1024, s, A, A, A, B, ws, None, None) == 1          # null W
+    assert f(A, A, A, 1, 3000, 1024, s, A, A, A, None, ws, None, None) == 1          # null workspace
+    assert f(A, A, A, 1, 3000, 40, s, A, A, A, B, ws, None, None) == 2               # C % 32
+    assert f(A, A, A, 5, 3000, 1024, s, A, A, A, B, ws, None, None) == 4             # dtype
+    assert f(A, A, A, 1, 3000, 1024, s, A, A, A, B, ws - 1, None, None) == 5         # small workspace
+    assert f(A, A, A, 1, 3000, 1024, s, A, A, A, ct.c_void_p(0x20010), ws, None, None) == 3  # alignment

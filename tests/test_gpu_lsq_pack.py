@@ -130,3 +130,22 @@ def test_lsq_pack_full_workloads(cfg, cache, oracle_mod):
     Q2, gW2, gD2 = q4.lsq_fwd_bwd(tW, tD, tG)
     torch.cuda.synchronize()
     assert torch.equal(Q, Q2) and torch.equal(gW, gW2) and torch.equal(gD, gD2)
+
+
+@pytest.mark.parametrize("R,C,gdt,pinned", [(3000, 1024, "bf16", True), (5000, 1024, "f32", True),
+                                           (70, 96, "bf16", False), (1, 32, "f32", True)])
+def test_lsq_fwd_bwd_host_matches_device_path(R, C, gdt, pinned):
+    """The host-buffer pipeline (row chunks uploaded, run and downloaded on two streams) gives the
+    same bits as the device call: 1 to 3 chunks, a ragged last chunk, pageable and pinned memory."""
+    W = inputs.student_t((R, C), 3.0, 0.01, seed=R, cfg=60, name="W")
+    d = (np.abs(W).reshape(R, C // 32, 32).max(axis=2) / np.float32(7)).astype(np.float32)
+    G = (np.random.default_rng(R).standard_normal((R, C)) * 1e-3).astype(np.float32)
+    Wt, dt = torch.from_numpy(W), torch.from_numpy(d)
+    Gt = torch.from_numpy(G).to(torch.bfloat16) if gdt == "bf16" else torch.from_numpy(G)
+    if pinned:
+        Wt, dt, Gt = Wt.pin_memory(), dt.pin_memory(), Gt.pin_memory()
+    Qh, gWh, gDh = q4.lsq_fwd_bwd_host(Wt, dt, Gt)
+    torch.cuda.current_stream().synchronize()
+    Qd, gWd, gDd = q4.lsq_fwd_bwd(Wt.cuda(), dt.cuda(), Gt.cuda())
+    q4.sync_check()
+    assert torch.equal(Qh, Qd.cpu()) and torch.equal(gWh, gWd.cpu()) and torch.equal(gDh, gDd.cpu())
