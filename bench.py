@@ -461,6 +461,160 @@ def run_reference(args):
     }), flush=True)
 
 
+def run_stack(args):
+    """A whole decoder stack: config 3 (1B-class, 16 layers, 112 matrices, every matrix searched,
+    64 calibration Hessians of n = 65536) or config 4 (8B-class, 32 layers, 224 matrices, layer 0's
+    4 Hessians of n = 131072 and 7 searches, RTN scales elsewhere).  A step is every Hessian, every
+    search, one fused LSQ step over every weight and the W4A16 export of every matrix; each stage's
+    launches (independent matrices) go round-robin to four streams and the stage is timed with CUDA
+    events on the launching stream, which waits for all four (every stage's inputs are far larger
+    than L2).  Inputs are drawn on the GPU with torch's CUDA generator (seed 0) with the workload's shapes
+    and distributions (weights N(0, sigma); X rows N(0, 1) with round(1% d) outlier channels x20,
+    rounded to bf16; G N(0, 1e-3) in bf16); parity at these shapes is covered by the workload tests
+    on the host-seeded tensors.  One JSON line."""
+    import torch
+
+    import int4_group_wise_b200 as q4
+    from int4_group_wise_b200 import inputs
+
+    if args.config not in (3, 4):
+        raise SystemExit("--variant stack runs config 3 or 4")
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    peaks, peak_kind = load_peaks()
+    wl = inputs.workload(args.config)
+    gen = torch.Generator(device=dev).manual_seed(layer_seed(rank))
+    t0 = time.time()
+
+    def randn(shape, sigma):
+        return torch.randn(shape, generator=gen, device=dev, dtype=torch.float32).mul_(sigma)
+
+    X, H = {}, {}
+    for x_name, d in wl.calib.items():
+        x = torch.randn((wl.n_calib, d), generator=gen, device=dev, dtype=torch.float32)
+        cols = torch.randperm(d, generator=gen, device=dev)[:wl.outliers.get(x_name, 0)]
+        x[:, cols] *= 20.0
+        X[x_name] = x.to(torch.bfloat16)
+        del x
+        H[x_name] = torch.empty((d, d), dtype=torch.float32, device=dev)
+    ws = torch.empty(max([q4.hessian_workspace_bytes(wl.n_calib, d) for d in wl.calib.values()] + [16]),
+                     dtype=torch.uint8, device=dev)
+    alpha = torch.from_numpy(wl.alpha()).to(dev)
+    mats = []
+    for m in wl.matrices:
+        W = randn((m.d_out, m.d_in), wl.weight_sigma)
+        G = randn((m.d_out, m.d_in), 1e-3).to(torch.bfloat16)
+        # scales of matrices that are not searched: round-to-nearest (alpha = 1), fl(max|w_g| / 7)
+        delta = (W.abs().view(m.d_out, m.d_in // 32, 32).amax(-1) / 7.0).contiguous()
+        mats.append(dict(m=m, W=W, G=G, delta=delta, idx=torch.empty(delta.shape, dtype=torch.int32, device=dev),
+                         err=torch.empty_like(delta), Q=torch.empty_like(W), gW=torch.empty_like(W),
+                         gD=torch.empty_like(delta),
+                         packed=torch.empty((m.d_out, m.d_in // 2), dtype=torch.uint8, device=dev),
+                         scales=torch.empty(delta.shape, dtype=torch.float16, device=dev)))
+    gen_s = time.time() - t0
+    searched = [e for e in mats if e["m"].name in wl.searched]
+    n_weights = sum(e["W"].numel() for e in mats)
+    hess_flop = sum(float(wl.n_calib) * d * (d + 1) for d in wl.calib.values())
+    groups = sum(e["W"].numel() // 32 for e in searched)
+    K = int(alpha.numel())
+    stream = torch.cuda.current_stream(dev)
+    # independent matrices go round-robin to NS side streams (the small k/v launches alone leave
+    # most SMs idle); each stage starts after the previous one on every stream and ends when all
+    # side streams are done; each stream has its own Hessian workspace
+    NS = 4
+    side = [torch.cuda.Stream(device=dev) for _ in range(NS)]
+    wss = [ws] + [torch.empty_like(ws) for _ in range(NS - 1)]
+
+    def fan(launches):
+        go = torch.cuda.Event()
+        go.record(stream)
+        for s_ in side:
+            s_.wait_event(go)
+        for i, launch in enumerate(launches):
+            with torch.cuda.stream(side[i % NS]):
+                launch(i % NS)
+        for s_ in side:
+            done = torch.cuda.Event()
+            done.record(s_)
+            stream.wait_event(done)
+
+    def stage_hessian():
+        fan([lambda j, x=x_name: q4.hessian(X[x], H[x], wss[j]) for x_name in wl.calib])
+
+    def stage_search():
+        fan([lambda j, e=e: q4.scale_search(e["W"], H[e["m"].x_name], alpha, e["delta"], e["idx"], e["err"])
+             for e in searched])
+
+    def stage_lsq():
+        fan([lambda j, e=e: q4.lsq_fwd_bwd(e["W"], e["delta"], e["G"], q4.GRAD_SCALE, e["Q"], e["gW"], e["gD"])
+             for e in mats])
+
+    def stage_pack():
+        fan([lambda j, e=e: q4.pack_w4a16(e["W"], e["delta"], e["packed"], e["scales"]) for e in mats])
+
+    stages = [("hessian", stage_hessian), ("scale_search", stage_search), ("lsq_fwd_bwd", stage_lsq),
+              ("pack_w4a16", stage_pack)]
+
+    def step(ev=None):
+        for i, (_, fn) in enumerate(stages):
+            if ev is not None:
+                ev[i][0].record(stream)
+            fn()
+            if ev is not None:
+                ev[i][1].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    q4.sync_check()
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in stages] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"bench_stack_clocks_r{rank}.csv")) as clk:
+        start.record(stream)
+        for k in range(args.steps):
+            step(evs[k])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    q4.sync_check()
+    total_ms = start.elapsed_time(stop) / args.steps
+    mean = {name: sum(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(args.steps)) / args.steps
+            for i, (name, _) in enumerate(stages)}
+    hbm = float(peaks["hbm_gbs"])
+    tc_peak = float(peaks["bf16_tflops"])
+    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+    search_roof = 148 * 128 * sm_max * 1e6 / (SEARCH_OPS_PER_CAND * K)
+    lsq_bytes = LSQ_BYTES_PER_ELT * n_weights
+    pack_bytes = PACK_BYTES_PER_ELT * n_weights
+    lsq_gbs = lsq_bytes / mean["lsq_fwd_bwd"] / 1e6
+    st = {
+        "hessian": {"value": hess_flop / mean["hessian"] / 1e9, "unit": "TFLOP/s", "ms": mean["hessian"],
+                    "launches": len(wl.calib), "flop": hess_flop,
+                    "frac": hess_flop / mean["hessian"] / 1e9 / tc_peak},
+        "scale_search": {"value": groups / mean["scale_search"] * 1e3, "unit": "groups/s",
+                         "ms": mean["scale_search"], "launches": len(searched), "groups": groups,
+                         "frac": groups / mean["scale_search"] * 1e3 / search_roof},
+        "lsq_fwd_bwd": {"value": lsq_gbs, "unit": "GB/s", "ms": mean["lsq_fwd_bwd"], "launches": len(mats),
+                        "bytes": lsq_bytes, "frac": lsq_gbs / hbm},
+        "pack_w4a16": {"value": pack_bytes / mean["pack_w4a16"] / 1e6, "unit": "GB/s", "ms": mean["pack_w4a16"],
+                       "launches": len(mats), "bytes": pack_bytes,
+                       "frac": pack_bytes / mean["pack_w4a16"] / 1e6 / hbm},
+    }
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": lsq_gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "variant": "stack", "dtype": "f32", "data": "synthetic (drawn on the GPU)",
+            "config": {"workload": wl.title, "config_index": args.config, "matrices": len(mats),
+                       "weights": n_weights, "hessians": len(wl.calib), "n_calib": wl.n_calib,
+                       "searched_matrices": len(searched), "K": K,
+                       "streams": NS, "l2": "every stage's inputs are larger than L2; no flush"},
+            "stages": st, "peaks": {"hbm_gbs": hbm, "bf16_tflops": tc_peak, "kind": peak_kind,
+                                    "search_roof_groups_per_s": search_roof},
+            "gpu_launches": (len(wl.calib) * 2 + len(searched) + 2 * len(mats)) * args.steps,
+            "clocks": clk.summary(), "input_gen_s": round(gen_s, 1)}), flush=True)
+
+
 def run_per_channel(args):
     """The per-channel variant (one scale per row) on the same layer shape: fused LSQ step and
     W4A16 export, each launch timed with CUDA events after an L2 flush; one JSON line."""
@@ -898,13 +1052,14 @@ def main():
     ap.add_argument("--config", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--variant", choices=["group32", "per-channel", "w4a16-decode", "fq-gemm", "hessian-split",
-                                          "refine"],
+                                          "refine", "stack"],
                     default="group32",
                     help="per-channel: time the one-scale-per-row LSQ step and export instead; "
                          "w4a16-decode: time the inference GEMV on the packed 8B-class stack; "
                          "fq-gemm: time the fused fake-quant forward GEMM; "
                          "hessian-split: the calibration Hessian with its rows split over the ranks; "
-                         "refine: one sweep of the full-objective refinement")
+                         "refine: one sweep of the full-objective refinement; "
+                         "stack: the whole decoder stack of --config 3 or 4")
     ap.add_argument("--tokens", type=int, default=8192, help="fq-gemm: tokens of the micro-batch")
     ap.add_argument("--layers", type=int, default=None,
                     help="w4a16-decode: number of layers of the 8B-class stack (default: all 32)")
@@ -923,6 +1078,8 @@ def main():
         run_hessian_split(args)
     elif args.variant == "refine":
         run_refine(args)
+    elif args.variant == "stack":
+        run_stack(args)
     else:
         run_ours(args)
 
