@@ -137,38 +137,44 @@ __device__ __noinline__ void tc_error_exact(const float* __restrict__ wrow, floa
 // Start of row i of the row-major upper triangle (j >= i) of a 32x32 matrix.
 __host__ __device__ constexpr int tri_start(int i) { return 32 * i - (i * (i - 1)) / 2; }
 
-// float64 value of one candidate (the re-score): codes with the IEEE division,
-// Q = fl(dk * q), the exact difference e = w - Q (exact in binary64), and
-// e H' e summed in binary64 over the upper triangle H' (H'_ij = H_ij + H_ji,
-// H'_ii = H_ii).  Two rows at a time, each row's sum split in two, so four
-// independent FMA chains are in flight.
+// float64 value of one candidate (the re-score): the exact codes (w * (1/dk),
+// with the IEEE division redone for the group near a rounding boundary or when
+// 1/dk is not finite, as in the screen), Q = fl(dk * q), the exact difference
+// e = w - Q (exact in binary64), and e H' e summed in binary64 over the upper
+// triangle H' (H'_ij = H_ij + H_ji, H'_ii = H_ii).  Four rows at a time, each
+// row's sum split in two, so eight independent FMA chains are in flight.
 __device__ __forceinline__ double tc_quad_form64(const double* h64, const float (&w)[32], float dk) {
     double ed[32];
+    const float rc = __frcp_rn(dk);
+    float fmax_abs = 0.0f;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-        const float q = code_of(scaled_exact(w[i], dk));
+        const float x = fminf(fmaxf(__fmul_rn(w[i], rc), kQmin), kQmax);
+        const float q = __fsub_rn(__fadd_rn(x, kMagic), kMagic);
+        fmax_abs = fmaxf(fmax_abs, fabsf(__fsub_rn(x, q)));
         ed[i] = static_cast<double>(w[i]) - static_cast<double>(__fmul_rn(dk, q));
     }
-    double E0 = 0.0, E1 = 0.0;
+    if (!(fmax_abs <= kTieWindow && fabsf(rc) <= 3.4028234663852886e38f)) {
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-        double ta = 0.0, tb = 0.0, tc = 0.0, td = 0.0;
-        const double* ra = h64 + tri_start(i);          // row i: j = i..31
-        const double* rb = h64 + tri_start(i + 1);      // row i + 1: j = i + 1..31
-#pragma unroll
-        for (int j = i; j < 32; ++j) {
-            if ((j - i) & 1) tb = fma(ra[j - i], ed[j], tb);
-            else ta = fma(ra[j - i], ed[j], ta);
+        for (int i = 0; i < 32; ++i) {
+            const float q = code_of(scaled_exact(w[i], dk));
+            ed[i] = static_cast<double>(w[i]) - static_cast<double>(__fmul_rn(dk, q));
         }
-#pragma unroll
-        for (int j = i + 1; j < 32; ++j) {
-            if ((j - i - 1) & 1) td = fma(rb[j - i - 1], ed[j], td);
-            else tc = fma(rb[j - i - 1], ed[j], tc);
-        }
-        E0 = fma(ed[i], ta + tb, E0);
-        E1 = fma(ed[i + 1], tc + td, E1);
     }
-    return E0 + E1;
+    double E[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+        double t[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const double* row = h64 + tri_start(i + r);     // row i + r: j = i + r..31
+#pragma unroll
+            for (int j = i + r; j < 32; ++j) t[2 * r + ((j - i - r) & 1)] = fma(row[j - i - r], ed[j], t[2 * r + ((j - i - r) & 1)]);
+        }
+#pragma unroll
+        for (int r = 0; r < 4; ++r) E[r] = fma(ed[i + r], t[2 * r] + t[2 * r + 1], E[r]);
+    }
+    return (E[0] + E[1]) + (E[2] + E[3]);
 }
 
 // Quantizes one candidate for this thread's row: writes e_hi into the stage's
@@ -353,8 +359,14 @@ scale_search_kernel(const float* __restrict__ W, int R, int C,
             }
         }
     }
-    atomicMax(&sm.kappa_bits, __float_as_uint(kap));
-    atomicMax(&sm.hmax_bits, __float_as_uint(hmax));
+    {   // non-negative floats order like their bit patterns: one shared atomic per warp
+        const unsigned kb = __reduce_max_sync(0xffffffffu, __float_as_uint(kap));
+        const unsigned hb = __reduce_max_sync(0xffffffffu, __float_as_uint(hmax));
+        if ((tid & 31) == 0) {
+            atomicMax(&sm.kappa_bits, kb);
+            atomicMax(&sm.hmax_bits, hb);
+        }
+    }
     __syncthreads();
 
     // scale of the block: 2^13 <= hmax * sigma_H < 2^14
@@ -389,7 +401,10 @@ scale_search_kernel(const float* __restrict__ W, int R, int C,
         *reinterpret_cast<__half*>(sm.bhi + off) = hi;
         *reinterpret_cast<__half*>(sm.blo + off) = lo;
     }
-    atomicMax(&sm.kappa_d_bits, __float_as_uint(kapd));
+    {
+        const unsigned db = __reduce_max_sync(0xffffffffu, __float_as_uint(kapd));
+        if ((tid & 31) == 0) atomicMax(&sm.kappa_d_bits, db);
+    }
     __syncthreads();
     if (tid == 0) {
         const double kp = static_cast<double>(__uint_as_float(sm.kappa_bits));
