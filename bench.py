@@ -52,6 +52,8 @@ CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.a
 
 # --------------------------------------------------------------------------- setup
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_1b_up_proj.md")
+# where the nvidia-smi clock samples of the timed region are written (one CSV per rank)
+OUT_DIR = os.environ.get("QAT4_BENCH_OUT", os.path.join(ROOT, "bench_out"))
 STAGE_KERNELS = {"hessian": ["hessian_pair_kernel", "hessian_reduce_kernel"],
                  "scale_search": ["scale_search_kernel"], "lsq_fwd_bwd": ["lsq_blocks_kernel"],
                  "pack_w4a16": ["pack_w4a16_blocks_kernel"]}
@@ -156,6 +158,7 @@ class ClockSampler:
                 out, _ = self.proc.communicate()
             self.lines = [ln for ln in out.splitlines() if ln.strip()]
             if self.out_path:
+                os.makedirs(os.path.dirname(self.out_path), exist_ok=True)
                 with open(self.out_path, "w") as fh:
                     fh.write(CLOCK_FIELDS + "\n" + "\n".join(self.lines) + "\n")
 
@@ -255,11 +258,11 @@ def run_ours(args):
 
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in stages] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    os.makedirs(os.path.join(ROOT, "gpurun_out"), exist_ok=True)
+    os.makedirs(OUT_DIR, exist_ok=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"bench_clocks_r{rank}.csv")) as clk:
+    with ClockSampler(local, os.path.join(OUT_DIR, f"bench_clocks_r{rank}.csv")) as clk:
         start.record(stream)
         for k in range(args.steps):
             step(evs[k])
@@ -570,7 +573,7 @@ def run_stack(args):
     evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in stages] for _ in range(args.steps)]
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
-    with ClockSampler(local, os.path.join(ROOT, "gpurun_out", f"bench_stack_clocks_r{rank}.csv")) as clk:
+    with ClockSampler(local, os.path.join(OUT_DIR, f"bench_stack_clocks_r{rank}.csv")) as clk:
         start.record(stream)
         for k in range(args.steps):
             step(evs[k])
