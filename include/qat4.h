@@ -179,7 +179,10 @@ qat4_status qat4_lsq_fwd_bwd(const float *W, const float *delta, const void *G, 
  *            `stream` has completed (cudaStreamSynchronize), the outputs are
  *            on the host.  copy_stream may equal stream (then nothing overlaps).
  *  The call creates and releases five CUDA events per call; it allocates no
- *  memory.  Errors: QAT4_ERR_NULL, _SHAPE, _DTYPE, _WORKSPACE, _ALIGN, _CUDA.
+ *  memory.  Errors: QAT4_ERR_NULL, _SHAPE, _DTYPE, _WORKSPACE, _ALIGN (all
+ *  before anything is enqueued) and _CUDA (a copy, launch or event call
+ *  failed; the outputs are then incomplete, and `stream` still waits for the
+ *  copies that were enqueued).
  */
 size_t qat4_lsq_fwd_bwd_host_workspace_bytes(int64_t R, int64_t C, qat4_dtype g_dtype);
 qat4_status qat4_lsq_fwd_bwd_host(const float *W, const float *delta, const void *G, qat4_dtype g_dtype,

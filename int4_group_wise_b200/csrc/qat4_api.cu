@@ -338,13 +338,13 @@ qat4_status qat4_lsq_fwd_bwd_host(const float* W, const float* delta, const void
         buf[b].d = reinterpret_cast<float*>(p);            p += r256(n / 32 * 4);
         buf[b].gd = reinterpret_cast<float*>(p);
     }
-    cudaEvent_t done[2], freed[2], last;
+    cudaEvent_t done[2] = {nullptr, nullptr}, freed[2] = {nullptr, nullptr}, last = nullptr;
     bool made = true;
     for (int b = 0; b < 2; ++b) {
-        made &= cudaEventCreateWithFlags(&done[b], cudaEventDisableTiming) == cudaSuccess;
-        made &= cudaEventCreateWithFlags(&freed[b], cudaEventDisableTiming) == cudaSuccess;
+        made = made && cudaEventCreateWithFlags(&done[b], cudaEventDisableTiming) == cudaSuccess;
+        made = made && cudaEventCreateWithFlags(&freed[b], cudaEventDisableTiming) == cudaSuccess;
     }
-    made &= cudaEventCreateWithFlags(&last, cudaEventDisableTiming) == cudaSuccess;
+    made = made && cudaEventCreateWithFlags(&last, cudaEventDisableTiming) == cudaSuccess;
     qat4_status st = made ? QAT4_OK : QAT4_ERR_CUDA;
     const auto H2D = cudaMemcpyHostToDevice;
     const auto D2H = cudaMemcpyDeviceToHost;
@@ -373,16 +373,17 @@ qat4_status qat4_lsq_fwd_bwd_host(const float* W, const float* delta, const void
         ok &= cudaEventRecord(freed[b], copy_stream) == cudaSuccess;
         if (!ok) st = QAT4_ERR_CUDA;
     }
-    // completion is observable on `stream`: it waits for the last download
-    if (made) {
-        if (cudaEventRecord(last, copy_stream) != cudaSuccess || cudaStreamWaitEvent(stream, last, 0) != cudaSuccess)
-            st = QAT4_ERR_CUDA;
-        for (int b = 0; b < 2; ++b) {
-            cudaEventDestroy(done[b]);
-            cudaEventDestroy(freed[b]);
-        }
-        cudaEventDestroy(last);
+    // completion is observable on `stream`: it waits for the last download (also after an error
+    // part-way, so that nothing of this call is still running when `stream` has completed)
+    if (made && (cudaEventRecord(last, copy_stream) != cudaSuccess ||
+                 cudaStreamWaitEvent(stream, last, 0) != cudaSuccess))
+        st = QAT4_ERR_CUDA;
+    // release whatever was created (destruction of a pending event is deferred by the runtime)
+    for (int b = 0; b < 2; ++b) {
+        if (done[b]) cudaEventDestroy(done[b]);
+        if (freed[b]) cudaEventDestroy(freed[b]);
     }
+    if (last) cudaEventDestroy(last);
     return st;
 }
 
