@@ -374,7 +374,9 @@ def run_ours(args):
                     "what": "lsq_fwd_bwd_host (C ABI qat4_lsq_fwd_bwd_host) from pinned host W, G, delta to "
                             "pinned host Q, grad_W, grad_delta: row chunks of ~2 M weights, uploads on the "
                             "compute stream overlapping downloads on a copy stream"},
-            "gpu_launches": 4 * args.steps,
+            # per step: Hessian pair kernel (+ the reduction of split partials when n is split),
+            # search, fused LSQ, pack
+            "gpu_launches": (4 + (1 if ws_bytes > 0 else 0)) * args.steps,
             "clocks": clocks,
             "input_gen_s": round(gen_s, 1),
         }
