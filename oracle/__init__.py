@@ -29,6 +29,7 @@ def lib():
         L.oracle_hessian.argtypes = [_P, _I64, _I64, _P]
         L.oracle_hessian_entries.argtypes = [_P, _I64, _I64, _P, _P, _I64, _P]
         L.oracle_hessian_block.argtypes = [_P, _I64, _I64, _I64, _I64, _I64, _I64, _P]
+        L.oracle_hessian_blocks.argtypes = [_P, _I64, _I64, _P, _P, _I64, _I64, _P]
         L.oracle_scale_search.argtypes = [_P, _I64, _I64, _P, _I64, _P, ct.c_int32, _P, _P, _P, _P]
         L.oracle_lsq_fwd.argtypes = [_P, _P, _I64, _I64, _P]
         L.oracle_lsq_bwd.argtypes = [_P, _P, _P, ct.c_int, _I64, _I64, ct.c_float, _P, _P]
@@ -39,7 +40,7 @@ def lib():
         L.oracle_pack_w4a16_rowwise.argtypes = [_P, _P, _I64, _I64, _P, _P]
         L.oracle_scale_search_rowwise.argtypes = [_P, _I64, _I64, _P, _I64, _P, ct.c_int32, _P, _P, _P, _P]
         L.oracle_w4a16_gemv.argtypes = [_P, _P, _P, _I64, _I64, _I64, _I64, _P]
-        for f in ("oracle_hessian", "oracle_hessian_entries", "oracle_hessian_block",
+        for f in ("oracle_hessian", "oracle_hessian_entries", "oracle_hessian_block", "oracle_hessian_blocks",
                   "oracle_scale_search", "oracle_lsq_fwd", "oracle_lsq_bwd",
                   "oracle_pack_w4a16", "oracle_codes", "oracle_lsq_fwd_rowwise",
                   "oracle_lsq_bwd_rowwise", "oracle_pack_w4a16_rowwise", "oracle_scale_search_rowwise",
@@ -85,6 +86,19 @@ def hessian_block(X_bits: np.ndarray, r0: int, nr: int, c0: int, nc: int) -> np.
     n, C = X.shape
     out = np.empty((nr, nc), np.float64)
     lib().oracle_hessian_block(_p(X), n, C, r0, nr, c0, nc, _p(out))
+    return out
+
+
+def hessian_blocks(X_bits: np.ndarray, r0, c0, b: int) -> np.ndarray:
+    """Blocks H[r0[m]:r0[m]+b, c0[m]:c0[m]+b] in float64, shape [count, b, b] (one block per thread)."""
+    X = _c(X_bits, np.uint16)
+    n, C = X.shape
+    r0 = _c(r0, np.int64)
+    c0 = _c(c0, np.int64)
+    assert r0.shape == c0.shape and r0.ndim == 1 and 0 < b <= 256
+    assert np.all((r0 >= 0) & (r0 + b <= C) & (c0 >= 0) & (c0 + b <= C))
+    out = np.empty((r0.size, b, b), np.float64)
+    lib().oracle_hessian_blocks(_p(X), n, C, _p(r0), _p(c0), r0.size, b, _p(out))
     return out
 
 

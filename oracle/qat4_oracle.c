@@ -110,17 +110,20 @@ static float fake_quant(float w, float delta)
  * X: bf16 bits, row-major [n, C].  H: double, row-major [C, C] (full). */
 void oracle_hessian(const uint16_t *X, int64_t n, int64_t C, double *H)
 {
+    /* Row i of H is one accumulator per column j; the calibration rows t are
+     * visited in order, so every entry is the sum over t = 0, 1, ..., n-1
+     * taken left to right, starting from 0. */
     #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t i = 0; i < C; ++i) {
-        for (int64_t j = 0; j < C; ++j) {
-            double s = 0.0;
-            for (int64_t t = 0; t < n; ++t) {
-                double xi = (double)bf16_to_float(X[t * C + i]);
-                double xj = (double)bf16_to_float(X[t * C + j]);
-                s += xi * xj;
-            }
-            H[i * C + j] = s / (double)n;
+        double *s = H + i * C;
+        for (int64_t j = 0; j < C; ++j) s[j] = 0.0;
+        for (int64_t t = 0; t < n; ++t) {
+            const uint16_t *xt = X + t * C;
+            const double xi = (double)bf16_to_float(xt[i]);
+            for (int64_t j = 0; j < C; ++j)
+                s[j] += xi * (double)bf16_to_float(xt[j]);
         }
+        for (int64_t j = 0; j < C; ++j) s[j] = s[j] / (double)n;
     }
 }
 
@@ -142,22 +145,55 @@ void oracle_hessian_entries(const uint16_t *X, int64_t n, int64_t C,
     }
 }
 
+/* One block H[r0:r0+nr, c0:c0+nc] into out (row-major [nr, nc]), computed by
+ * the calling thread: for every calibration row t in order, every entry of the
+ * block adds x[t][r0+a] * x[t][c0+b].  Same sums, same order as
+ * oracle_hessian. */
+static void hessian_block_serial(const uint16_t *X, int64_t n, int64_t C,
+                                 int64_t r0, int64_t nr, int64_t c0, int64_t nc, double *out)
+{
+    double xb[256];                       /* x[t][c0 .. c0+nc-1], nc <= 256 */
+    for (int64_t m = 0; m < nr * nc; ++m) out[m] = 0.0;
+    for (int64_t t = 0; t < n; ++t) {
+        const uint16_t *xt = X + t * C;
+        for (int64_t b = 0; b < nc; ++b) xb[b] = (double)bf16_to_float(xt[c0 + b]);
+        for (int64_t a = 0; a < nr; ++a) {
+            const double xa = (double)bf16_to_float(xt[r0 + a]);
+            double *s = out + a * nc;
+            for (int64_t b = 0; b < nc; ++b)
+                s[b] += xa * xb[b];
+        }
+    }
+    for (int64_t m = 0; m < nr * nc; ++m) out[m] = out[m] / (double)n;
+}
+
 /* A dense block H[r0:r0+nr, c0:c0+nc] (row-major [nr, nc] in out). */
 void oracle_hessian_block(const uint16_t *X, int64_t n, int64_t C,
                           int64_t r0, int64_t nr, int64_t c0, int64_t nc, double *out)
 {
+    /* one strip of 8 rows by up to 256 columns of the block per thread */
+    const int64_t strips = (nr + 7) / 8, panels = (nc + 255) / 256;
     #pragma omp parallel for schedule(dynamic, 1)
-    for (int64_t a = 0; a < nr; ++a) {
-        for (int64_t b = 0; b < nc; ++b) {
-            double s = 0.0;
-            for (int64_t t = 0; t < n; ++t) {
-                double xi = (double)bf16_to_float(X[t * C + r0 + a]);
-                double xj = (double)bf16_to_float(X[t * C + c0 + b]);
-                s += xi * xj;
-            }
-            out[a * nc + b] = s / (double)n;
-        }
+    for (int64_t sp = 0; sp < strips * panels; ++sp) {
+        const int64_t a = (sp / panels) * 8, b = (sp % panels) * 256;
+        const int64_t rows = (nr - a < 8) ? nr - a : 8;
+        const int64_t cols = (nc - b < 256) ? nc - b : 256;
+        double tmp[8 * 256];
+        hessian_block_serial(X, n, C, r0 + a, rows, c0 + b, cols, tmp);
+        for (int64_t i = 0; i < rows; ++i)
+            for (int64_t j = 0; j < cols; ++j) out[(a + i) * nc + b + j] = tmp[i * cols + j];
     }
+}
+
+/* Many b x b blocks (b <= 256): block m is H[r0[m]:r0[m]+b, c0[m]:c0[m]+b],
+ * written to out + m*b*b (row-major).  One block per thread. */
+void oracle_hessian_blocks(const uint16_t *X, int64_t n, int64_t C,
+                           const int64_t *r0, const int64_t *c0, int64_t count, int64_t b,
+                           double *out)
+{
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t m = 0; m < count; ++m)
+        hessian_block_serial(X, n, C, r0[m], b, c0[m], b, out + m * b * b);
 }
 
 /* ------------------------------------------ (b) Hessian-weighted scale search

@@ -1,12 +1,14 @@
 """GPU parity of the calibration Hessian against the float64 oracle:
 relative Frobenius error <= 1e-3 (tensor-core fp32 accumulation of exact
-bf16 products), bitwise symmetry, and run-to-run determinism."""
+bf16 products) over the whole matrix AND over every checked 32x32 block on
+its own (hessian_check), bitwise symmetry, and run-to-run determinism."""
 import numpy as np
 import pytest
 import torch
 
 import int4_group_wise_b200 as q4
 from int4_group_wise_b200 import inputs
+from hessian_check import check_blocks, check_hessian
 
 pytestmark = pytest.mark.gpu
 f32 = np.float32
@@ -23,6 +25,13 @@ def _frob(a, b):
     return float(np.linalg.norm(a.astype(np.float64) - b) / np.linalg.norm(b))
 
 
+def _every_block(Hg, Hr):
+    """Each 32x32 block of a fully computed H within 1e-3 relative Frobenius error on its own."""
+    C = Hr.shape[0]
+    starts = [(r, c) for r in range(0, C, 32) for c in range(0, C, 32)]
+    check_blocks(Hg, np.stack([Hr[r:r + 32, c:c + 32] for r, c in starts]), starts, 32)
+
+
 @pytest.mark.parametrize("n,C", [(1, 32), (63, 32), (65, 96), (200, 160), (64, 128), (129, 256),
                                  (1000, 288), (4096, 384)])
 def test_hessian_small(n, C, oracle_mod):
@@ -31,6 +40,7 @@ def test_hessian_small(n, C, oracle_mod):
     Hg = H.cpu().numpy()
     Hr = oracle_mod.hessian(Xb)
     assert _frob(Hg, Hr) <= 1e-3
+    _every_block(Hg, Hr)
     np.testing.assert_array_equal(Hg, Hg.T)
     assert np.all(np.isfinite(Hg))
 
@@ -51,6 +61,7 @@ def test_hessian_config0_full_and_deterministic(cache, oracle_mod):
     Hr = oracle_mod.hessian(Xb)
     Hg = H.cpu().numpy()
     assert _frob(Hg, Hr) <= 1e-3
+    _every_block(Hg, Hr)
     np.testing.assert_array_equal(Hg, Hg.T)
     H2 = q4.hessian(X)
     torch.cuda.synchronize()
@@ -58,29 +69,20 @@ def test_hessian_config0_full_and_deterministic(cache, oracle_mod):
 
 
 @pytest.mark.parametrize("cfg", [1, 2])
-def test_hessian_full_size_sampled(cfg, cache, oracle_mod):
-    """Full n x C on the GPU; the oracle recomputes every 32x32 diagonal block
-    plus seeded random 128x128 tiles (upper and lower), Frobenius over the sample."""
+def test_hessian_full_size_every_tile(cfg, cache, oracle_mod):
+    """Full n x C on the GPU (config 1: C = 2048, 36 upper tiles, n split in two and the
+    partials reduced; config 2: C = 8192, 528 upper tiles stored directly).  The oracle
+    recomputes every 32x32 diagonal block, one seeded 32x32 block inside every upper-triangle
+    256x256 tile, and seeded random 128x128 tiles (64 at config 2) anywhere in H; each block
+    must be within 1e-3 relative Frobenius error on its own."""
     wl = inputs.workload(cfg)
     Xb = cache.get(("X", cfg, "x"), lambda: wl.activations("x"))
     X, H = _gpu_h(Xb)
     Hg = H.cpu().numpy()
-    C = Xb.shape[1]
+    del X, H
     np.testing.assert_array_equal(Hg, Hg.T)
-    num = den = 0.0
-    for g in range(C // 32):
-        ref = oracle_mod.hessian_block(Xb, 32 * g, 32, 32 * g, 32)
-        got = Hg[32 * g:32 * g + 32, 32 * g:32 * g + 32]
-        num += float(np.sum((got - ref) ** 2))
-        den += float(np.sum(ref ** 2))
-    rng = np.random.default_rng(cfg)
-    for _ in range(4):
-        r0, c0 = (int(v) * 128 for v in rng.integers(0, C // 128, 2))
-        ref = oracle_mod.hessian_block(Xb, r0, 128, c0, 128)
-        got = Hg[r0:r0 + 128, c0:c0 + 128]
-        num += float(np.sum((got - ref) ** 2))
-        den += float(np.sum(ref ** 2))
-    assert (num / den) ** 0.5 <= 1e-3, (num / den) ** 0.5
+    assert np.all(np.isfinite(Hg))
+    check_hessian(Hg, Xb, oracle_mod, np.random.default_rng(cfg), n_random=64 if cfg == 2 else 16)
 
 
 @pytest.mark.parametrize("n,C", [(40000, 3072), (50000, 2048), (20000, 512)])
@@ -91,16 +93,7 @@ def test_hessian_multi_chunk_ragged(n, C, oracle_mod):
     X, H = _gpu_h(Xb)
     Hg = H.cpu().numpy()
     np.testing.assert_array_equal(Hg, Hg.T)
-    rng = np.random.default_rng(n)
-    num = den = 0.0
-    blocks = [(0, 0), (C - 128, C - 128)] + [tuple(int(v) * 64 for v in rng.integers(0, C // 64 - 1, 2))
-                                             for _ in range(3)]
-    for r0, c0 in blocks:
-        ref = oracle_mod.hessian_block(Xb, r0, 128 if r0 + 128 <= C else 64, c0, 128 if c0 + 128 <= C else 64)
-        got = Hg[r0:r0 + ref.shape[0], c0:c0 + ref.shape[1]]
-        num += float(np.sum((got - ref) ** 2))
-        den += float(np.sum(ref ** 2))
-    assert (num / den) ** 0.5 <= 1e-3, (num / den) ** 0.5
+    check_hessian(Hg, Xb, oracle_mod, np.random.default_rng(n), n_random=6)
 
 
 def test_hessian_workspace_contract():

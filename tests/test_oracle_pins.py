@@ -212,6 +212,40 @@ def test_hessian_entries_and_block_consistent(oracle_mod):
     np.testing.assert_array_equal(oracle_mod.hessian_block(Xb, 32, 32, 0, 64), H[32:64, 0:64])
 
 
+def test_hessian_blocks_closed_forms(oracle_mod):
+    """The batched block call (used by the full-size GPU checks) against closed forms that do not
+    form X^T X: a bilinear form u^T H_blk v = (X_r u) . (X_c v) / n from two matrix-vector
+    products, the one-hot diagonal case, and the hand 2x2 case inside a larger matrix."""
+    rng = np.random.default_rng(9)
+    n, C = 300, 192
+    Xb = _bf16(rng.standard_normal((n, C)) * np.linspace(0.3, 4, C))
+    X = inputs.bf16_bits_to_f32(Xb).astype(np.float64)
+    r0 = [0, 32, 160, 96]
+    c0 = [64, 32, 0, 128]
+    blocks = oracle_mod.hessian_blocks(Xb, r0, c0, 32)
+    for b, r, c in zip(blocks, r0, c0):
+        for _ in range(3):
+            u, v = rng.standard_normal(32), rng.standard_normal(32)
+            lhs = u @ b @ v
+            rhs = (X[:, r:r + 32] @ u) @ (X[:, c:c + 32] @ v) / n
+            assert abs(lhs - rhs) <= 1e-12 * (np.abs(X[:, r:r + 32] @ np.abs(u)) @ np.abs(X[:, c:c + 32] @ np.abs(v)) / n)
+    # one-hot rows: every off-diagonal block is exactly zero, diagonal blocks are diag(sum a_t^2)/n
+    cols = rng.integers(0, C, 64)
+    a = rng.choice([-2.0, 0.5, 1.0, 3.0], 64)
+    Xo = np.zeros((64, C), f32)
+    Xo[np.arange(64), cols] = a
+    bo = oracle_mod.hessian_blocks(_bf16(Xo), [0, 64, 32], [32, 64, 160], 32)
+    assert not bo[0].any() and not bo[2].any()
+    exp = np.zeros(C)
+    np.add.at(exp, cols, a ** 2)
+    np.testing.assert_array_equal(bo[1], np.diag(exp[64:96] / 64))
+    # hand 2x2 case [[1, 2], [3, 4]] placed in columns 40, 41 of zeros: H[40:42, 40:42] = [[5, 7], [7, 10]]
+    Xh = np.zeros((2, 96), f32)
+    Xh[:, 40:42] = [[1, 2], [3, 4]]
+    bh = oracle_mod.hessian_blocks(_bf16(Xh), [32], [32], 32)[0]
+    np.testing.assert_array_equal(bh[8:10, 8:10], [[5.0, 7.0], [7.0, 10.0]])
+
+
 # --------------------------------------------------------------- scale search
 
 def _integer_calibration(rng, n, C):
