@@ -218,7 +218,12 @@ qat4_status qat4_pack_w4a16(const float *W, const float *delta, int64_t R, int64
  *              QAT4_ERR_WORKSPACE.
  *  The call allocates nothing: no cudaMalloc, cudaFree or allocating library
  *  routine.  Its first call on a device (with that device current) looks up
- *  the array's device address once; make that first call before any stream
+ *  the array's device address once and keeps it; make that first call before
+ *  any stream capture.  The kept address belongs to the device's context: the
+ *  call compares the current context's id (cuCtxGetId) with the one the
+ *  address was looked up in, and after cudaDeviceReset, whose next CUDA call
+ *  runs in a new context, it looks the address up again -- so the first call
+ *  after a reset is again a set-up call and must also come before any
  *  capture.  All calls on a device share the one array: two calls whose
  *  kernels overlap on the GPU (different streams, or other host threads)
  *  race on it and must be ordered by the caller.  Every byte of the scratch

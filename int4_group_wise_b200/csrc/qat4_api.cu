@@ -35,6 +35,7 @@ bool valid_rc(int64_t R, int64_t C) {
 }
 
 struct DeviceInfo {
+    unsigned long long ctx_id = 0;   // context the cached set-up below belongs to
     int sms = 0;
     bool hessian_attr = false;
     bool search_attr = false;
@@ -45,12 +46,50 @@ struct DeviceInfo {
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mutex;
 
-// Current device and its SM count (cached); false on any CUDA error.
+// Unique id of the calling thread's current CUDA context (the driver never
+// reuses one within a process), or 0 if it cannot be read.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+unsigned long long current_ctx_id() {
+    static std::once_flag once;
+    static CtxGetCurrentFn get_current = nullptr;
+    static CtxGetIdFn get_id = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<CtxGetIdFn>(p);
+    });
+    if (!get_current || !get_id) return 0;
+    CUcontext c = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&c) != CUDA_SUCCESS || c == nullptr || get_id(c, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Current device and its cached set-up (SM count, kernel attributes); false on
+// any CUDA error.  The set-up is tied to the device's context: when the context
+// has changed since it was made (cudaDeviceReset destroys the primary context,
+// and the next call runs in a new one), it is dropped and made again.
 bool device_info(int* dev_out, DeviceInfo** info) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+    unsigned long long ctx = current_ctx_id();
+    if (ctx == 0) {   // no context current yet: cudaSetDevice creates and binds it
+        if (cudaSetDevice(dev) != cudaSuccess) return false;
+        ctx = current_ctx_id();
+    }
     std::lock_guard<std::mutex> lock(g_mutex);
     DeviceInfo& d = g_dev[dev];
+    if (ctx != 0 && ctx != d.ctx_id) {
+        d = DeviceInfo{};
+        d.ctx_id = ctx;
+    }
     if (d.sms == 0) {
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
@@ -737,7 +776,8 @@ constexpr size_t kNoallocScratchBytes =
 
 static __device__ __align__(256) unsigned char g_hessian_scratch[kNoallocScratchBytes];
 
-void* g_scratch_addr[kMaxDevices] = {};   // device address of g_hessian_scratch, per device
+void* g_scratch_addr[kMaxDevices] = {};              // device address of g_hessian_scratch
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // the context that address belongs to
 
 }  // namespace
 
@@ -748,17 +788,21 @@ extern "C" qat4_status qat4_hessian_noalloc(const uint16_t* X, int64_t n, int64_
     const size_t need = qat4_hessian_workspace_bytes(n, C);
     if (need > kNoallocScratchBytes) return QAT4_ERR_WORKSPACE;   // larger than the built-in scratch
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QAT4_ERR_CUDA;
+    DeviceInfo* info = nullptr;
+    if (!device_info(&dev, &info)) return QAT4_ERR_CUDA;           // also makes the context current
+    const unsigned long long ctx = current_ctx_id();
     void* scratch = nullptr;
     {
-        // One-time set-up per device, with that device current: host code only
-        // knows a stand-in for the array, so its device address is looked up.
+        // Set-up once per device (and again if its context has been replaced, as after
+        // cudaDeviceReset), with that device current: host code only knows a stand-in
+        // for the array, so its device address is looked up.
         std::lock_guard<std::mutex> lock(g_mutex);
-        if (g_scratch_addr[dev] == nullptr) {
+        if (g_scratch_addr[dev] == nullptr || ctx == 0 || ctx != g_scratch_ctx[dev]) {
             void* addr = nullptr;
             if (cudaGetSymbolAddress(&addr, g_hessian_scratch) != cudaSuccess || addr == nullptr)
                 return QAT4_ERR_CUDA;
             g_scratch_addr[dev] = addr;
+            g_scratch_ctx[dev] = ctx;
         }
         scratch = g_scratch_addr[dev];
     }

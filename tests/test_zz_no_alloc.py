@@ -13,6 +13,7 @@ import torch
 
 import int4_group_wise_b200 as q4
 from int4_group_wise_b200 import inputs
+from hessian_check import check_hessian
 
 pytestmark = pytest.mark.gpu
 
@@ -28,7 +29,7 @@ def _frob(a, b):
     return float(torch.linalg.norm((a - b).double()) / torch.linalg.norm(b.double()))
 
 
-def test_noalloc_matches_workspace_entry_point_twice_in_a_row():
+def test_noalloc_matches_workspace_entry_point_twice_in_a_row(oracle_mod):
     # a shape whose n is split, so the scratch is really used (18 MiB at 65536 x 2048 would also do)
     n, C = 8192, 1024
     assert q4.hessian_workspace_bytes(n, C) > 0
@@ -44,6 +45,8 @@ def test_noalloc_matches_workspace_entry_point_twice_in_a_row():
         q4.sync_check()
         assert _frob(H_noalloc, H_ref) <= 1e-3
         assert torch.equal(H_noalloc, H_ref)      # same kernels, same order: identical bits
+        # and against the float64 oracle, block by block over every upper tile
+        check_hessian(H_noalloc.cpu().numpy(), Xb, oracle_mod, np.random.default_rng(seed), n_random=4)
         results.append(H_noalloc)
     assert not torch.equal(results[0], results[1])
 
