@@ -1,24 +1,31 @@
 """Benchmark of the group-32 INT4 quantizer path on B200.
 
-One step = one pass of the whole path over one 1B-class MLP up-projection
-(W fp32 8192x2048, calibration X bf16 262144x2048 with 1% outlier channels,
-101-candidate grid, upstream gradient bf16):
+One step = one pass of the whole path over a workload, inputs resident in HBM:
 
-    H = hessian(X) -> (delta, idx, err) = scale_search(W, H, alpha)
-      -> (Q, grad_W, grad_delta) = lsq_fwd_bwd(W, delta, G) -> pack_w4a16(W, delta)
+    H = hessian(X) for every calibration input
+      -> (delta, idx, err) = scale_search(W, H, alpha) for every searched matrix
+      -> (Q, grad_W, grad_delta) = lsq_fwd_bwd(W, delta, G) for every matrix
+      -> (packed, scales) = pack_w4a16(W, delta) for every matrix
 
-Every input is resident in HBM before timing starts.  Before each stage the
-L2 cache (126 MB) is flushed by a read sweep over a 512 MB buffer, so no
-stage reads its inputs from L2; the flushes are inside ms_per_step but not
-inside the per-kernel times.  Per-kernel times are CUDA events on the stream
-the kernels run on.
+The headline step is the 8B-class decoder stack (hidden 4096, MLP 14336, 32
+layers, 224 matrices, 6.98 G fp32 weights): layer 0's four calibration
+Hessians from 131072 rows, layer 0's seven scale searches over the
+101-candidate grid, one fused LSQ step over all 224 matrices (99.5 GB moved)
+and the W4A16 export of all 224 (the largest configuration that fits one
+GPU).  Each stage's launches go round-robin to four streams; every stage's
+inputs are larger than L2.  After it, the 1B-class MLP up-projection
+(8192x2048, X 262144x2048) and the heavy-tailed down-projection (2048x8192,
+X 262144x8192, 201 candidates) are timed the same way, one launch per stage,
+with L2 flushed before every stage, and reported under `stages.config1` and
+`stages.config2`.  Per-stage times are CUDA events on the launching stream.
 
 The headline `value` is the first metric of the path, LSQ fwd+bwd GB/s
 (14.25 algorithmic bytes per weight); the Hessian TFLOP/s, scale-search
 groups/s and pack GB/s are in `stages`, each with its roofline.  With N GPUs
-every rank quantizes its own layer (independent problems, weak scaling, no
-collective on the data path); the value is the bytes of all ranks divided by
-the slowest rank's time.
+every rank runs its own seeded copy of the workload (independent problems,
+weak scaling, no collective on the data path); the value is the bytes of all
+ranks divided by the slowest rank's time.  `--gpus N` started without a
+launcher re-executes itself under torch.distributed.run with N ranks.
 
 `--impl reference` times the CPU oracle instead (test infrastructure, run
 only here and in the tests) on a bounded sample of the same workload.
@@ -41,6 +48,7 @@ if ROOT not in sys.path:
 
 METRIC = "LSQ fwd+bwd GB/s (% HBM peak); scale-search groups/s; Hessian TFLOP/s"
 LSQ_BYTES_PER_ELT = 14.25       # W 4 + G(bf16) 2 + Q 4 + grad_W 4 + (delta 4 + grad_delta 4)/32
+LSQ_BYTES_PER_ELT_F32G = 16.25  # the same with an fp32 G
 PACK_BYTES_PER_ELT = 4.6875     # W 4 + delta 4/32 + nibbles 0.5 + fp16 scale 2/32
 SEARCH_OPS_PER_CAND = 720       # 528 FMA quadratic form + 32 x (div, rint, min, max, mul, sub)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
@@ -51,14 +59,12 @@ CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.a
 
 
 # --------------------------------------------------------------------------- setup
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_1b_up_proj.md")
-# where the nvidia-smi clock samples of the timed region are written (one CSV per rank)
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic_path.md")
+# where the nvidia-smi clock samples of the timed regions are written (one CSV per config and rank)
 OUT_DIR = os.environ.get("QAT4_BENCH_OUT", os.path.join(ROOT, "bench_out"))
 STAGE_KERNELS = {"hessian": ["hessian_pair_kernel", "hessian_reduce_kernel"],
                  "scale_search": ["scale_search_kernel"], "lsq_fwd_bwd": ["lsq_blocks_kernel"],
                  "pack_w4a16": ["pack_w4a16_blocks_kernel"]}
-
-
 STEP_SOURCES = ("device_common.cuh", "hessian.cuh", "lsq_pack.cuh", "scale_search.cuh")
 
 
@@ -75,21 +81,27 @@ def source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def load_traffic(config: int):
-    """Per-stage DRAM bytes per launch from the committed ncu table, or {} when stale or absent."""
-    if config != 1 or not os.path.exists(TRAFFIC_FILE):
+def load_traffic(config: int, p=None):
+    """Per-stage DRAM bytes per step from the committed table of ncu captures.
+
+    The table holds, per configuration and kernel, dram__bytes_read.sum + dram__bytes_write.sum
+    summed over the launches of one step, with the sources' hash at capture time.  It is a stored
+    figure: a stage gets {"bytes", "source"} only while the kernel sources still hash to the
+    recorded value, and nothing (null in the line) after any change to them."""
+    if not os.path.exists(TRAFFIC_FILE):
         return {}
     text = open(TRAFFIC_FILE).read()
     recorded = next((ln.split(":", 1)[1].strip() for ln in text.splitlines() if ln.startswith("source_hash:")), None)
-    if recorded != source_hash():
+    if recorded is None or recorded != source_hash():
         return {}
-    per_kernel = {}
+    per = {}
     for ln in text.splitlines():
         f = [x.strip() for x in ln.strip().strip("|").split("|")]
-        if len(f) == 2 and f[1].isdigit():
-            per_kernel[f[0]] = int(f[1])
-    return {st: sum(per_kernel.get(k, 0) for k in ks) for st, ks in STAGE_KERNELS.items()
-            if all(k in per_kernel for k in ks)}
+        if len(f) == 3 and f[0].isdigit() and f[2].isdigit():
+            per[(int(f[0]), f[1])] = int(f[2])
+    src = f"stored ncu capture ({os.path.relpath(TRAFFIC_FILE, ROOT)}, source hash {recorded})"
+    return {st: {"bytes": sum(per[(config, k)] for k in ks if (config, k) in per), "source": src}
+            for st, ks in STAGE_KERNELS.items() if (config, ks[0]) in per}
 
 
 def load_peaks():
@@ -106,6 +118,18 @@ def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", str(rank)))
     return rank, world, local
+
+
+def relaunch_ranks(n: int, argv) -> int:
+    """Runs this script as n ranks on this node under torch.distributed.run (rendezvous on
+    127.0.0.1, a free port); returns the launcher's exit status."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__), *argv]
+    return subprocess.run(cmd).returncode
 
 
 def layer_seed(rank: int) -> int:
@@ -182,206 +206,341 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------------ device workloads
+class DeviceProblem:
+    """One workload drawn on the GPU with torch's CUDA generator: every matrix's W (fp32,
+    N(0, sigma) or Student-t(3) * 0.01), G (N(0, 1e-3); bf16, fp32 for the small layer), its
+    scales (the search writes those of the searched matrices; the others get round-to-nearest
+    scales fl(max|w_g| / 7)) and outputs, and per distinct layer input the calibration X (rows
+    N(0, 1), round(1% d) outlier channels x20 or lognormal channel scales, rounded to bf16) and
+    H.  Host-generating the 8B-class stack (28 GB of weights) would dominate the run; parity at
+    these shapes is covered by the tests on the host-seeded tensors."""
+
+    def __init__(self, cfg: int, dev, seed: int, q4, streams: int):
+        import torch
+        from int4_group_wise_b200 import inputs
+        self.cfg = cfg
+        self.wl = wl = inputs.workload(cfg)
+        self.dev = dev
+        gen = torch.Generator(device=dev).manual_seed(1000 * cfg + seed)
+        randn = lambda shape: torch.randn(shape, generator=gen, device=dev, dtype=torch.float32)
+        t0 = time.time()
+        self.X, self.H = {}, {}
+        for x_name, d in wl.calib.items():
+            x = randn((wl.n_calib, d))
+            scale = torch.ones(d, device=dev)
+            k = wl.outliers.get(x_name) or 0
+            if k:
+                scale[torch.randperm(d, generator=gen, device=dev)[:k]] = 20.0
+            if wl.lognormal_channels:
+                scale *= randn((d,)).exp_()
+            x *= scale
+            self.X[x_name] = x.to(torch.bfloat16)
+            del x
+            self.H[x_name] = torch.empty((d, d), dtype=torch.float32, device=dev)
+        self.n_ws = max([q4.hessian_workspace_bytes(wl.n_calib, d) for d in wl.calib.values()] + [16])
+        self.ws = [torch.empty(self.n_ws, dtype=torch.uint8, device=dev) for _ in range(streams)]
+        self.alpha = torch.from_numpy(wl.alpha()).to(dev)
+        self.mats = []
+        for m in wl.matrices:
+            shape = (m.d_out, m.d_in)
+            if wl.weight_student_t:
+                chi2 = randn(shape).square_()
+                chi2 += randn(shape).square_()
+                chi2 += randn(shape).square_()
+                W = randn(shape).div_(chi2.div_(3.0).sqrt_()).mul_(0.01)
+                del chi2
+            else:
+                W = randn(shape).mul_(wl.weight_sigma)
+            G = randn(shape).mul_(1e-3)
+            if wl.g_dtype == "bf16":
+                G = G.to(torch.bfloat16)
+            delta = (W.abs().view(m.d_out, m.d_in // 32, 32).amax(-1) / 7.0).contiguous()
+            self.mats.append(dict(
+                m=m, W=W, G=G, delta=delta, idx=torch.empty(delta.shape, dtype=torch.int32, device=dev),
+                err=torch.empty_like(delta), Q=torch.empty_like(W), gW=torch.empty_like(W),
+                gD=torch.empty_like(delta), packed=torch.empty((m.d_out, m.d_in // 2), dtype=torch.uint8, device=dev),
+                scales=torch.empty(delta.shape, dtype=torch.float16, device=dev)))
+        torch.cuda.synchronize(dev)
+        self.gen_s = time.time() - t0
+        self.searched = [e for e in self.mats if e["m"].name in wl.searched]
+        self.weights = sum(e["W"].numel() for e in self.mats)
+        self.hess_flop = sum(float(wl.n_calib) * d * (d + 1) for d in wl.calib.values())
+        self.groups = sum(e["W"].numel() // 32 for e in self.searched)
+        self.K = int(self.alpha.numel())
+        self.lsq_bpe = LSQ_BYTES_PER_ELT if wl.g_dtype == "bf16" else LSQ_BYTES_PER_ELT_F32G
+        # kernel launches of one step: a Hessian is one launch, plus the reduction of its
+        # partials when its calibration rows are split
+        self.launches = (sum(1 + (q4.hessian_workspace_bytes(wl.n_calib, d) > 0) for d in wl.calib.values())
+                         + len(self.searched) + 2 * len(self.mats))
+
+    def units(self):
+        return {"hessian": self.hess_flop, "scale_search": float(self.groups),
+                "lsq_fwd_bwd": self.lsq_bpe * self.weights, "pack_w4a16": PACK_BYTES_PER_ELT * self.weights}
+
+
+STAGES = ("hessian", "scale_search", "lsq_fwd_bwd", "pack_w4a16")
+
+
+def time_problem(p: DeviceProblem, q4, steps: int, warmup: int, flush: bool, world: int, rank: int,
+                 local: int, clock_name: str | None):
+    """Warm-up, then exactly `steps` steps bracketed by a barrier and a device synchronize on both
+    sides.  A step runs the four stages over every matrix of the workload: each stage's launches
+    (independent matrices) go round-robin to side streams (one launch goes on the launching
+    stream itself), the stage ends when all are done, and CUDA events on the launching stream
+    bracket it.  With `flush`, a 512 MB read sweep evicts L2 before every stage (inside the step
+    time, outside the stage times)."""
+    import torch
+    import torch.distributed as dist
+    dev = p.dev
+    stream = torch.cuda.current_stream(dev)
+    ns = len(p.ws)
+    side = [torch.cuda.Stream(device=dev) for _ in range(ns)] if ns > 1 else []
+    flush_buf = torch.ones(128 << 20, dtype=torch.float32, device=dev) if flush else None
+    sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def fan(launches):
+        if not side:
+            for launch in launches:
+                launch(0)
+            return
+        go = torch.cuda.Event()
+        go.record(stream)
+        for s_ in side:
+            s_.wait_event(go)
+        for i, launch in enumerate(launches):
+            with torch.cuda.stream(side[i % ns]):
+                launch(i % ns)
+        for s_ in side:
+            done = torch.cuda.Event()
+            done.record(s_)
+            stream.wait_event(done)
+
+    stage_fn = {
+        "hessian": lambda: fan([lambda j, x=x: q4.hessian(p.X[x], p.H[x], p.ws[j]) for x in p.wl.calib]),
+        "scale_search": lambda: fan([lambda j, e=e: q4.scale_search(e["W"], p.H[e["m"].x_name], p.alpha, e["delta"],
+                                                                    e["idx"], e["err"]) for e in p.searched]),
+        "lsq_fwd_bwd": lambda: fan([lambda j, e=e: q4.lsq_fwd_bwd(e["W"], e["delta"], e["G"], q4.GRAD_SCALE, e["Q"],
+                                                                  e["gW"], e["gD"]) for e in p.mats]),
+        "pack_w4a16": lambda: fan([lambda j, e=e: q4.pack_w4a16(e["W"], e["delta"], e["packed"], e["scales"])
+                                   for e in p.mats]),
+    }
+
+    def step(ev=None):
+        for i, name in enumerate(STAGES):
+            if flush:
+                torch.sum(flush_buf, dim=0, out=sink)
+            if ev is not None:
+                ev[i][0].record(stream)
+            stage_fn[name]()
+            if ev is not None:
+                ev[i][1].record(stream)
+
+    for _ in range(warmup):
+        step()
+    q4.sync_check()
+    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in STAGES] for _ in range(steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    path = os.path.join(OUT_DIR, f"{clock_name}_r{rank}.csv") if clock_name else None
+    with ClockSampler(local, path) as clk:
+        start.record(stream)
+        for k in range(steps):
+            step(evs[k])
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    q4.sync_check()
+    mean = {s: sum(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(steps)) / steps
+            for i, s in enumerate(STAGES)}
+    del flush_buf
+    return {"total_ms": start.elapsed_time(stop), "stage_ms": mean, "clocks": clk.summary()}
+
+
+def stage_lines(p: DeviceProblem, res, world: int, peaks, peak_kind: str, long_step: bool, traffic: dict):
+    """Per-stage whole-job rate and roofline: units of all ranks / the slowest rank's time.
+    Every rank makes the same collective calls in the same order."""
+    units = p.units()
+    job = {s: aggregate_over_ranks(units[s], res["stage_ms"][s]) for s in STAGES}
+    hbm = float(peaks["hbm_gbs"])
+    burst = float(peaks["bf16_tflops"])
+    sustained = float(peaks.get("bf16_tflops_sustained", burst))
+    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
+    alu_peak = 148 * 128 * sm_max * 1e6                                  # FP32 ops/s, one per lane per clock
+    search_roof = alu_peak / (SEARCH_OPS_PER_CAND * p.K)                 # groups/s
+    tc = sustained if long_step else burst
+    out = {}
+    u, ms = job["hessian"]
+    v = u / ms / 1e9
+    out["hessian"] = {"value": v, "unit": "TFLOP/s", "ms": ms, "launches": len(p.wl.calib),
+                      "roofline": {"bound": "tensor", "achieved": v / world, "peak": tc, "unit": "TFLOP/s",
+                                   "frac": v / world / tc, "frac_of_burst": v / world / burst,
+                                   "frac_of_sustained": v / world / sustained,
+                                   "algorithmic_per_step": units["hessian"],
+                                   "peak_kind": f"{peak_kind} bf16 {'sustained' if long_step else 'burst'}"}}
+    u, ms = job["scale_search"]
+    v = u / ms * 1e3
+    out["scale_search"] = {"value": v, "unit": "groups/s", "ms": ms, "launches": len(p.searched), "K": p.K,
+                           "roofline": {"bound": "alu", "achieved": v / world * SEARCH_OPS_PER_CAND * p.K / 1e12,
+                                        "peak": alu_peak / 1e12, "unit": "Top/s", "frac": v / world / search_roof,
+                                        "ops_per_group": SEARCH_OPS_PER_CAND * p.K, "groups_per_step": units["scale_search"],
+                                        "peak_kind": f"148 SM x 128 FP32 lanes x {sm_max:.0f} MHz"}}
+    for s in ("lsq_fwd_bwd", "pack_w4a16"):
+        u, ms = job[s]
+        v = u / ms / 1e6
+        out[s] = {"value": v, "unit": "GB/s", "ms": ms, "launches": len(p.mats),
+                  "roofline": {"bound": "hbm", "achieved": v / world, "peak": hbm, "unit": "GB/s",
+                               "frac": v / world / hbm, "bytes_per_step": units[s], "peak_kind": f"{peak_kind} copy"}}
+    for s in STAGES:
+        t = traffic.get(s)
+        out[s]["roofline"]["traffic"] = t["bytes"] if t else None
+        if t:
+            out[s]["roofline"]["traffic_source"] = t["source"]
+    return out
+
+
+def e2e_lsq_stack(p: DeviceProblem, q4, steps: int):
+    """The LSQ step of the stack end to end through the host-buffer call qat4_lsq_fwd_bwd_host:
+    each call uploads W, G and the scales from page-locked host memory, runs the fused kernel on
+    row chunks and downloads Q, grad_W and grad_delta (uploads on the caller's stream overlap the
+    downloads on a copy stream).  Layer 0's seven matrices are held on the host (3 GB page-locked)
+    and stand in for every layer of the stack, so one e2e step moves the whole stack's bytes
+    through PCIe.  Returns (ms per step, h2d bytes, d2h bytes, algorithmic bytes)."""
+    import torch
+    dev = p.dev
+    layer0 = [e for e in p.mats if e["m"].name.startswith("L0.")] if p.cfg in (3, 4) else p.mats
+    reps = len(p.mats) // len(layer0)
+    host = []
+    for e in layer0:
+        h = {k: e[k].cpu().pin_memory() for k in ("W", "G", "delta")}
+        h.update(Q=torch.empty(e["W"].shape, dtype=torch.float32).pin_memory(),
+                 gW=torch.empty(e["W"].shape, dtype=torch.float32).pin_memory(),
+                 gD=torch.empty(e["delta"].shape, dtype=torch.float32).pin_memory())
+        host.append(h)
+    gd = q4.QAT4_BF16 if p.wl.g_dtype == "bf16" else q4.QAT4_F32
+    ws = torch.empty(max(q4.lsq_fwd_bwd_host_workspace_bytes(*e["W"].shape, gd) for e in layer0),
+                     dtype=torch.uint8, device=dev)
+    cs = torch.cuda.Stream(device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def one():
+        for _ in range(reps):
+            for h in host:
+                q4.lsq_fwd_bwd_host(h["W"], h["delta"], h["G"], q4.GRAD_SCALE, h["Q"], h["gW"], h["gD"],
+                                    workspace=ws, copy_stream=cs)
+
+    one()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        one()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    q4.sync_check()
+    ms = a.elapsed_time(b) / steps
+    gbytes = 2 if gd == q4.QAT4_BF16 else 4
+    h2d = reps * sum(h["W"].numel() * (4 + gbytes) + h["delta"].numel() * 4 for h in host)
+    d2h = reps * sum(h["W"].numel() * 8 + h["delta"].numel() * 4 for h in host)
+    return ms, h2d, d2h, p.lsq_bpe * p.weights
+
+
+def cpu_model() -> str:
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+        for ln in out.splitlines():
+            if ln.lower().startswith("model name"):
+                return ln.split(":", 1)[1].strip()
+    except (OSError, subprocess.SubprocessError):
+        pass
+    return "unknown"
+
+
 # ------------------------------------------------------------------------ our arm
+PATH_CONFIGS = (4, 1, 2)        # the headline step first, then the single-layer configurations
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
 
     import int4_group_wise_b200 as q4
-    from int4_group_wise_b200 import inputs
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
         from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=dev)
     peaks, peak_kind = load_peaks()
-
-    wl = inputs.workload(args.config)
-    m = wl.matrices[0]
-    seed = layer_seed(rank)
-    t0 = time.time()
-    W_h = wl.weight(m, seed)
-    X_h = wl.activations(m.x_name, seed)
-    G_h = wl.grad(m, seed)
-    alpha_h = wl.alpha()
-    gen_s = time.time() - t0
-    R, C = W_h.shape
-    n = X_h.shape[0]
-    groups = R * C // 32
-    K = alpha_h.size
-
-    # pinned host copies (for the end-to-end leg) and device-resident inputs
-    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
-    W_p, X_p, G_p, a_p = pin(W_h), pin(X_h.view(np.int16)), pin(G_h.view(np.int16)), pin(alpha_h)
-    W = W_p.to(dev)
-    X = X_p.to(dev).view(torch.bfloat16)
-    G = G_p.to(dev).view(torch.bfloat16)
-    alpha = a_p.to(dev)
-    H = torch.empty((C, C), dtype=torch.float32, device=dev)
-    ws_bytes = q4.hessian_workspace_bytes(n, C)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
-    delta = torch.empty((R, C // 32), dtype=torch.float32, device=dev)
-    idx = torch.empty((R, C // 32), dtype=torch.int32, device=dev)
-    err = torch.empty((R, C // 32), dtype=torch.float32, device=dev)
-    Q = torch.empty_like(W)
-    gW = torch.empty_like(W)
-    gD = torch.empty_like(delta)
-    packed = torch.empty((R, C // 2), dtype=torch.uint8, device=dev)
-    scales = torch.empty((R, C // 32), dtype=torch.float16, device=dev)
-    flush_buf = torch.ones(128 << 20, dtype=torch.float32, device=dev)   # 512 MB
-    flush_sink = torch.empty((), dtype=torch.float32, device=dev)
-    stream = torch.cuda.current_stream(dev)
-
-    def flush():
-        torch.sum(flush_buf, dim=0, out=flush_sink)
-
-    stages = ["hessian", "scale_search", "lsq_fwd_bwd", "pack_w4a16"]
-
-    def step(ev=None):
-        def run(i, fn):
-            flush()
-            if ev is not None:
-                ev[i][0].record(stream)
-            fn()
-            if ev is not None:
-                ev[i][1].record(stream)
-        run(0, lambda: q4.hessian(X, H, ws))
-        run(1, lambda: q4.scale_search(W, H, alpha, delta, idx, err))
-        run(2, lambda: q4.lsq_fwd_bwd(W, delta, G, q4.GRAD_SCALE, Q, gW, gD))
-        run(3, lambda: q4.pack_w4a16(W, delta, packed, scales))
-
-    for _ in range(args.warmup):
-        step()
-    q4.sync_check()
-
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in stages] for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     os.makedirs(OUT_DIR, exist_ok=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local, os.path.join(OUT_DIR, f"bench_clocks_r{rank}.csv")) as clk:
-        start.record(stream)
-        for k in range(args.steps):
-            step(evs[k])
-        stop.record(stream)
-        torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    q4.sync_check()
-    total_ms = start.elapsed_time(stop)
-    per = {s: [evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(args.steps)] for i, s in enumerate(stages)}
-    mean = {s: sum(v) / len(v) for s, v in per.items()}
+    configs = PATH_CONFIGS if args.config is None else (args.config,)
+    seed = layer_seed(rank)
+    results = {}
+    for i, cfg in enumerate(configs):
+        stack = cfg in (3, 4)
+        p = DeviceProblem(cfg, dev, seed, q4, streams=4 if stack else 1)
+        res = time_problem(p, q4, args.steps, args.warmup, flush=not stack, world=world, rank=rank, local=local,
+                           clock_name=f"bench_clocks_c{cfg}")
+        job_steps, job_total = aggregate_over_ranks(1.0, res["total_ms"])
+        traffic = load_traffic(cfg, p)
+        lines = stage_lines(p, res, world, peaks, peak_kind, long_step=stack, traffic=traffic)
+        entry = {"workload": p.wl.title, "config_index": cfg, "ms_per_step": job_total / args.steps,
+                 "matrices": len(p.mats), "weights": p.weights, "hessians": len(p.wl.calib),
+                 "n_calib": p.wl.n_calib, "searched_matrices": len(p.searched), "K": p.K,
+                 "streams": len(p.ws), "stages": lines, "clocks": res["clocks"],
+                 "gpu_launches": p.launches * args.steps, "input_gen_s": round(p.gen_s, 1),
+                 "l2": ("every stage's inputs are larger than L2 (126 MB); no flush" if stack else
+                        "flushed (512 MB read sweep) before every stage; flush time in ms_per_step only")}
+        if i == 0 and not args.no_e2e:
+            ms, h2d, d2h, alg = e2e_lsq_stack(p, q4, steps=2 if stack else max(3, min(args.steps, 10)))
+            job_alg, job_ms = aggregate_over_ranks(alg, ms)
+            entry["e2e"] = {"value": job_alg / job_ms / 1e6, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                            "d2h_bytes_per_step": d2h, "ms_per_step": job_ms,
+                            "what": "the LSQ fwd+bwd step of the whole workload through the C ABI host-buffer "
+                                    "call qat4_lsq_fwd_bwd_host (page-locked host W, G, delta in; Q, grad_W, "
+                                    "grad_delta out; uploads overlap downloads)" +
+                                    ("; layer 0's seven host matrices stand in for every layer" if stack else "")}
+        if i == 0 and rank == 0 and world == 1 and not args.no_cpu_baseline:
+            entry["cpu_baseline"] = cpu_baseline(p)
+        results[cfg] = entry
+        del p
+        torch.cuda.empty_cache()
 
-    # ---- end-to-end leg: the host-buffer LSQ call (qat4_lsq_fwd_bwd_host) from pinned host
-    # memory and back; it streams row chunks through the GPU, uploads overlapping downloads
-    Q_p = torch.empty(Q.shape, dtype=Q.dtype).pin_memory()
-    gW_p = torch.empty(gW.shape, dtype=gW.dtype).pin_memory()
-    gD_p = torch.empty(gD.shape, dtype=gD.dtype).pin_memory()
-    d_p = delta.cpu().pin_memory()
-    G_pb = G_p.view(torch.bfloat16)
-    ws_host = torch.empty(q4.lsq_fwd_bwd_host_workspace_bytes(R, C, q4.QAT4_BF16), dtype=torch.uint8, device=dev)
-    copy_stream = torch.cuda.Stream(device=dev)
-
-    def e2e_step():
-        q4.lsq_fwd_bwd_host(W_p, d_p, G_pb, q4.GRAD_SCALE, Q_p, gW_p, gD_p, workspace=ws_host,
-                            copy_stream=copy_stream)
-
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    e2e_n = max(3, min(args.steps, 10))
-    a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a_.record(stream)
-    for _ in range(e2e_n):
-        e2e_step()
-    b_.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = a_.elapsed_time(b_) / e2e_n
-    h2d = W.numel() * 4 + G.numel() * 2 + delta.numel() * 4
-    d2h = Q.numel() * 4 + gW.numel() * 4 + gD.numel() * 4
-
-    # ---- whole-job aggregation (max time over ranks)
-    lsq_bytes = LSQ_BYTES_PER_ELT * R * C
-    job_lsq_bytes, job_lsq_ms = aggregate_over_ranks(lsq_bytes, mean["lsq_fwd_bwd"])
-    job_step_units, job_total_ms = aggregate_over_ranks(1.0, total_ms)
-    job_e2e_bytes, job_e2e_ms = aggregate_over_ranks(lsq_bytes, e2e_ms)
-    job_h_flop, job_h_ms = aggregate_over_ranks(float(n) * C * (C + 1), mean["hessian"])
-    job_groups, job_s_ms = aggregate_over_ranks(float(groups), mean["scale_search"])
-    job_pack_bytes, job_p_ms = aggregate_over_ranks(PACK_BYTES_PER_ELT * R * C, mean["pack_w4a16"])
-
+    head = results[configs[0]]
     if rank == 0:
-        clocks = clk.summary()
-        traffic = load_traffic(args.config)
-        hbm = float(peaks["hbm_gbs"])
-        tc_peak = float(peaks["bf16_tflops"])
-        sm_max = float(peaks.get("sm_max_mhz", 1965.0))
-        fp32_ops_peak = 148 * 128 * sm_max * 1e6            # one FP32 op per lane per clock
-        search_roof = fp32_ops_peak / (SEARCH_OPS_PER_CAND * K)   # groups/s, one GPU
-        lsq_gbs = job_lsq_bytes / job_lsq_ms / 1e6
-        stage_lines = {
-            "hessian": {"value": job_h_flop / job_h_ms / 1e9, "unit": "TFLOP/s", "ms": mean["hessian"],
-                        "roofline": {"bound": "tensor", "peak": tc_peak * world, "unit": "TFLOP/s",
-                                     "frac": job_h_flop / job_h_ms / 1e9 / (tc_peak * world),
-                                     "algorithmic_per_launch": float(n) * C * (C + 1),
-                                     "peak_kind": f"{peak_kind} bf16 burst"}},
-            "scale_search": {"value": job_groups / job_s_ms * 1e3, "unit": "groups/s", "ms": mean["scale_search"],
-                             "roofline": {"bound": "alu", "peak": search_roof * world, "unit": "groups/s",
-                                          "frac": job_groups / job_s_ms * 1e3 / (search_roof * world),
-                                          "ops_per_group": SEARCH_OPS_PER_CAND * K,
-                                          "peak_kind": f"148 SM x 128 FP32 lanes x {sm_max:.0f} MHz"}},
-            "lsq_fwd_bwd": {"value": lsq_gbs, "unit": "GB/s", "ms": mean["lsq_fwd_bwd"],
-                            "roofline": {"bound": "hbm", "peak": hbm * world, "unit": "GB/s",
-                                         "frac": lsq_gbs / (hbm * world), "bytes_per_launch": lsq_bytes,
-                                         "peak_kind": f"{peak_kind} copy"}},
-            "pack_w4a16": {"value": job_pack_bytes / job_p_ms / 1e6, "unit": "GB/s", "ms": mean["pack_w4a16"],
-                           "roofline": {"bound": "hbm", "peak": hbm * world, "unit": "GB/s",
-                                        "frac": job_pack_bytes / job_p_ms / 1e6 / (hbm * world),
-                                        "bytes_per_launch": PACK_BYTES_PER_ELT * R * C,
-                                        "peak_kind": f"{peak_kind} copy"}},
-        }
-        for st_name, line_st in stage_lines.items():
-            line_st["roofline"]["traffic"] = traffic.get(st_name)
-        dominant = max(stages, key=lambda s: mean[s])
-        dom = stage_lines[dominant]["roofline"]
-        if dominant == "hessian":
-            achieved, dom_peak = job_h_flop / job_h_ms / 1e9 / world, tc_peak
-        elif dominant == "scale_search":
-            achieved, dom_peak = job_groups / job_s_ms * 1e3 * SEARCH_OPS_PER_CAND * K / 1e12 / world, \
-                fp32_ops_peak / 1e12
-        else:
-            achieved = stage_lines[dominant]["value"] / world
-            dom_peak = hbm
-        roof_unit = {"hessian": "TFLOP/s", "scale_search": "Top/s"}.get(dominant, "GB/s")
+        st = head["stages"]
+        dominant = max(STAGES, key=lambda s: st[s]["ms"])
+        dom = st[dominant]["roofline"]
         line = {
-            "metric": METRIC, "value": lsq_gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": job_total_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": "1B-class MLP up-projection: W fp32 8192x2048, X bf16 262144x2048 "
-                                   "(1% outlier channels x20), 101-candidate grid, G bf16",
-                       "config_index": args.config, "R": R, "C": C, "n_calib": n, "K": K,
-                       "parallelism": f"replicas x{world} (one layer per GPU)",
-                       "l2": "flushed (512 MB read sweep) before every stage; flush time in ms_per_step only"},
-            "roofline": {"kernel": dominant, "bound": dom["bound"], "achieved": achieved, "peak": dom_peak,
-                         "unit": roof_unit, "frac": achieved / dom_peak,
-                         "traffic": traffic.get(dominant), "traffic_unit": "bytes per launch (ncu DRAM read + write)",
-                         "peak_kind": dom["peak_kind"]},
-            "stages": stage_lines,
-            "e2e": {"value": job_e2e_bytes / job_e2e_ms / 1e6, "unit": "GB/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "what": "lsq_fwd_bwd_host (C ABI qat4_lsq_fwd_bwd_host) from pinned host W, G, delta to "
-                            "pinned host Q, grad_W, grad_delta: row chunks of ~2 M weights, uploads on the "
-                            "compute stream overlapping downloads on a copy stream"},
-            # per step: Hessian pair kernel (+ the reduction of split partials when n is split),
-            # search, fused LSQ, pack
-            "gpu_launches": (4 + (1 if ws_bytes > 0 else 0)) * args.steps,
-            "clocks": clocks,
-            "input_gen_s": round(gen_s, 1),
+            "metric": METRIC, "value": st["lsq_fwd_bwd"]["value"], "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (drawn on the GPU with the workloads' distributions)",
+            "config": {"workload": head["workload"], "config_index": head["config_index"],
+                       "matrices": head["matrices"], "weights": head["weights"], "hessians": head["hessians"],
+                       "n_calib": head["n_calib"], "searched_matrices": head["searched_matrices"], "K": head["K"],
+                       "parallelism": f"replicas x{world} (every GPU its own seeded copy of the workload)",
+                       "l2": head["l2"]},
+            "roofline": {"kernel": dominant, **{k: dom[k] for k in ("bound", "achieved", "peak", "unit", "frac")},
+                         "traffic": dom.get("traffic"), "traffic_source": dom.get("traffic_source"),
+                         "traffic_unit": "bytes per step of the stage (ncu DRAM read + write)",
+                         "peak_kind": dom["peak_kind"],
+                         "note": "achieved = the stage's algorithmic work per step / its CUDA-event time "
+                                 "(launches fanned out over side streams, joined on the launching stream)"},
+            "stages": {**st, **{f"config{c}": {k: results[c][k] for k in
+                                               ("workload", "ms_per_step", "stages", "clocks", "gpu_launches", "l2")}
+                                for c in configs[1:]}},
+            "e2e": head.get("e2e"),
+            "gpu_launches": sum(results[c]["gpu_launches"] for c in configs),
+            "clocks": head["clocks"],
+            "input_gen_s": round(sum(results[c]["input_gen_s"] for c in configs), 1),
         }
-        if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(W_h, X_h, G_h, alpha_h)
+        if "cpu_baseline" in head:
+            line["cpu_baseline"] = head["cpu_baseline"]
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()
@@ -389,235 +548,150 @@ def run_ours(args):
 
 
 # ------------------------------------------------------------------ CPU oracle legs
-def _oracle_sample(W, X, G, alpha, rows: int, hblocks: int):
-    """One bounded sample of the step on the CPU oracle; returns per-stage (units, seconds)."""
+def _oracle_step(W, G, X, alpha, hblocks: int, search_rows: int):
+    """One pass of the oracle over host samples: LSQ fwd+bwd and pack over every matrix in W/G,
+    the diagonal 32x32 Hessian blocks 0..hblocks-1 of X over all its rows, and the scale search of
+    those groups on the first `search_rows` rows of the first matrix.  Returns per-stage
+    (units, seconds) in the GPU's units (flop, groups, bytes)."""
     import oracle
-    from int4_group_wise_b200.inputs import bf16_bits_to_f32  # noqa: F401  (inputs only)
     res = {}
-    Ws, Gs = W[:rows], G[:rows]
-    C = W.shape[1]
+    n = X.shape[0]
     t = time.perf_counter()
-    Hd = np.zeros((C, C), np.float32)
+    starts = [32 * g for g in range(hblocks)]
+    blocks = oracle.hessian_blocks(X, starts, starts, 32)
+    res["hessian"] = (float(n) * 32 * 33 * hblocks, time.perf_counter() - t)
+    Hd = np.zeros((32 * hblocks, 32 * hblocks), np.float32)
     for g in range(hblocks):
-        Hd[32 * g:32 * g + 32, 32 * g:32 * g + 32] = oracle.hessian_block(X, 32 * g, 32, 32 * g, 32)
-    res["hessian"] = (float(X.shape[0]) * 32 * 33 * hblocks, time.perf_counter() - t)
-    Wsearch = Ws[:, :32 * hblocks]
+        Hd[32 * g:32 * g + 32, 32 * g:32 * g + 32] = blocks[g]
+    Ws = np.ascontiguousarray(W[0][:search_rows, :32 * hblocks])
     t = time.perf_counter()
-    d, i, b = oracle.scale_search(Wsearch, Hd[:32 * hblocks, :32 * hblocks], alpha)
-    res["scale_search"] = (float(Wsearch.size // 32), time.perf_counter() - t)
-    delta = (np.abs(Ws).reshape(rows, -1, 32).max(axis=2) / np.float32(7)).astype(np.float32)
-    t = time.perf_counter()
-    oracle.lsq_fwd(Ws, delta)
-    oracle.lsq_bwd(Ws, delta, Gs, float(np.float32(1 / np.sqrt(224))))
-    res["lsq_fwd_bwd"] = (LSQ_BYTES_PER_ELT * Ws.size, time.perf_counter() - t)
-    t = time.perf_counter()
-    oracle.pack_w4a16(Ws, delta)
-    res["pack_w4a16"] = (PACK_BYTES_PER_ELT * Ws.size, time.perf_counter() - t)
+    oracle.scale_search(Ws, Hd, alpha)
+    res["scale_search"] = (float(Ws.size // 32), time.perf_counter() - t)
+    lsq_u = pack_u = lsq_s = pack_s = 0.0
+    s_ = float(np.float32(1 / np.sqrt(224)))
+    for w, g in zip(W, G):
+        delta = (np.abs(w).reshape(w.shape[0], -1, 32).max(axis=2) / np.float32(7)).astype(np.float32)
+        bpe = LSQ_BYTES_PER_ELT if g.dtype == np.uint16 else LSQ_BYTES_PER_ELT_F32G
+        t = time.perf_counter()
+        oracle.lsq_fwd(w, delta)
+        oracle.lsq_bwd(w, delta, g, s_)
+        lsq_s += time.perf_counter() - t
+        lsq_u += bpe * w.size
+        t = time.perf_counter()
+        oracle.pack_w4a16(w, delta)
+        pack_s += time.perf_counter() - t
+        pack_u += PACK_BYTES_PER_ELT * w.size
+    res["lsq_fwd_bwd"] = (lsq_u, lsq_s)
+    res["pack_w4a16"] = (pack_u, pack_s)
     return res
 
 
-def cpu_baseline(W, X, G, alpha, rows=2048, hblocks=8):
+def _rates(res):
+    return {"hessian_gflops": res["hessian"][0] / res["hessian"][1] * 1e-9,
+            "scale_search_groups_per_s": res["scale_search"][0] / res["scale_search"][1],
+            "lsq_fwd_bwd_gbs": res["lsq_fwd_bwd"][0] / res["lsq_fwd_bwd"][1] * 1e-9,
+            "pack_w4a16_gbs": res["pack_w4a16"][0] / res["pack_w4a16"][1] * 1e-9}
+
+
+def _host_bits(t):
+    """A device tensor as host NumPy data; bf16 as its uint16 bit patterns."""
+    import torch
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).cpu().numpy().view(np.uint16)
+    return t.cpu().numpy()
+
+
+def cpu_baseline(p: DeviceProblem, hblocks: int = 128):
+    """The oracle as it stands on the host cores, on a bounded sample of the workload the GPU
+    just ran (its own tensors, copied to the host): LSQ and pack over every matrix of layer 0 (for
+    the stacks; the whole layer otherwise), the first `hblocks` diagonal Hessian blocks over all
+    calibration rows of the first searched matrix's input, and the search of those groups over
+    all rows of that matrix."""
     import oracle
     cores = oracle.set_threads(0)
-    res = _oracle_sample(W, X, G, alpha, rows, hblocks)
-    u, s = res["lsq_fwd_bwd"]
-    return {"value": u / s / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"rows 0..{rows - 1} of W for LSQ/pack ({rows}x{W.shape[1]}); "
-                      f"{hblocks} diagonal 32x32 Hessian blocks over all {X.shape[0]} rows; "
-                      f"scale search on those {hblocks} groups x {rows} rows",
-            "stages": {"hessian_gflops": res["hessian"][0] * 1e-9 / res["hessian"][1] * 1.0,
-                       "scale_search_groups_per_s": res["scale_search"][0] / res["scale_search"][1],
-                       "lsq_fwd_bwd_gbs": u / s / 1e9,
-                       "pack_w4a16_gbs": res["pack_w4a16"][0] / res["pack_w4a16"][1] / 1e9}}
+    layer0 = [e for e in p.mats if e["m"].name.startswith("L0.")] if p.cfg in (3, 4) else p.mats
+    first = p.searched[0]
+    order = [first] + [e for e in layer0 if e is not first]
+    W = [_host_bits(e["W"]) for e in order]
+    G = [_host_bits(e["G"]) for e in order]
+    X = _host_bits(p.X[first["m"].x_name])
+    alpha = p.alpha.cpu().numpy()
+    hb = min(hblocks, X.shape[1] // 32)
+    rows = W[0].shape[0]
+    res = _oracle_step(W, G, X, alpha, hb, rows)
+    r = _rates(res)
+    return {"value": r["lsq_fwd_bwd_gbs"], "unit": "GB/s", "cores": cores, "cpu_model": cpu_model(),
+            "kind": "oracle",
+            "sample": (f"LSQ fwd+bwd and W4A16 pack over {'all 7 matrices of layer 0' if p.cfg in (3, 4) else 'the whole layer'} "
+                       f"({sum(w.size for w in W)} weights, in full); Hessian: {hb} diagonal 32x32 blocks of "
+                       f"{first['m'].x_name} over all {X.shape[0]} calibration rows (sampled); scale search: "
+                       f"those {hb} groups x {rows} rows of {first['m'].name} (sampled)"),
+            "seconds": round(sum(v[1] for v in res.values()), 2), "stages": r}
 
 
 def run_reference(args):
-    """The oracle as it stands, on the host cores, on bounded samples of the same workload."""
+    """The oracle as it stands on the host cores, on bounded samples of the headline workload:
+    each step runs every stage once on a fixed sample (the first rows of every layer-0 matrix for
+    LSQ and pack, diagonal Hessian blocks over a row sample of the calibration set, the search of
+    those groups on a row sample).  Under several ranks, rank 0 alone runs and prints; the others
+    exit without work."""
     rank, world, _ = dist_env()
-    if rank != 0:
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("gloo", timeout=timedelta(seconds=300))
+        try:
+            if rank == 0:
+                _reference_line(args, world)
+            dist.barrier()
+        finally:
+            dist.destroy_process_group()
         return
+    _reference_line(args, world)
+
+
+def _reference_line(args, world):
     import oracle
     from int4_group_wise_b200 import inputs
-    wl = inputs.workload(args.config)
-    m = wl.matrices[0]
-    W, G, alpha = wl.weight(m), wl.grad(m), wl.alpha()
-    X = wl.activations(m.x_name, n=16384)          # a row sample of the calibration set
+    cfg = 4 if args.config is None else args.config
+    wl = inputs.workload(cfg)
+    mats = [m for m in wl.matrices if m.name.startswith("L0.")] if cfg in (3, 4) else wl.matrices
+    rows = 256 if cfg in (3, 4) else 1024
+    searched = next(m for m in mats if m.name in wl.searched)
+    order = [searched] + [m for m in mats if m is not searched]
+    W = [wl.weight(m, rows=rows) for m in order]
+    G = [wl.grad(m, rows=rows) for m in order]
+    n = min(wl.n_calib, 16384)
+    X = wl.activations(searched.x_name, n=n)
+    alpha = wl.alpha()
+    hb = 4
     cores = oracle.set_threads(0)
-    rows = 512
     for _ in range(args.warmup):
-        _oracle_sample(W, X, G, alpha, rows, 2)
-    tot_u = tot_s = 0.0
+        _oracle_step(W, G, X, alpha, hb, rows)
+    tot = {s: [0.0, 0.0] for s in STAGES}
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        r = _oracle_sample(W, X, G, alpha, rows, 2)
-        tot_u += r["lsq_fwd_bwd"][0]
-        tot_s += r["lsq_fwd_bwd"][1]
+        r = _oracle_step(W, G, X, alpha, hb, rows)
+        for s in STAGES:
+            tot[s][0] += r[s][0]
+            tot[s][1] += r[s][1]
     wall = time.perf_counter() - t0
-    v = tot_u / tot_s / 1e9
-    sample = (f"per step: rows 0..{rows - 1} of W (LSQ, pack); 2 diagonal Hessian blocks over 16384 "
-              f"calibration rows; scale search on 2 groups x {rows} rows")
+    rates = _rates({s: tuple(v) for s, v in tot.items()})
+    v = rates["lsq_fwd_bwd_gbs"]
+    sample = (f"per step: the first {rows} rows of every {'layer-0 ' if cfg in (3, 4) else ''}matrix "
+              f"({sum(w.size for w in W)} weights) for LSQ fwd+bwd and pack; {hb} diagonal 32x32 Hessian blocks "
+              f"of {searched.x_name} over its first {n} calibration rows; the scale search of those {hb} groups "
+              f"x {rows} rows of {searched.name}")
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": v, "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": wall * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": "1B-class MLP up-projection (CPU oracle, row sample)", "config_index": args.config},
-        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "config": {"workload": f"{wl.title} (CPU oracle, bounded row sample)", "config_index": cfg},
+        "stages": rates,
+        "cpu_baseline": {"value": v, "unit": "GB/s", "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
+                         "sample": sample},
         "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
-
-
-def run_stack(args):
-    """A whole decoder stack: config 3 (1B-class, 16 layers, 112 matrices, every matrix searched,
-    64 calibration Hessians of n = 65536) or config 4 (8B-class, 32 layers, 224 matrices, layer 0's
-    4 Hessians of n = 131072 and 7 searches, RTN scales elsewhere).  A step is every Hessian, every
-    search, one fused LSQ step over every weight and the W4A16 export of every matrix; each stage's
-    launches (independent matrices) go round-robin to four streams and the stage is timed with CUDA
-    events on the launching stream, which waits for all four (every stage's inputs are far larger
-    than L2).  Inputs are drawn on the GPU with torch's CUDA generator (seed 0) with the workload's shapes
-    and distributions (weights N(0, sigma); X rows N(0, 1) with round(1% d) outlier channels x20,
-    rounded to bf16; G N(0, 1e-3) in bf16); parity at these shapes is covered by the workload tests
-    on the host-seeded tensors.  One JSON line."""
-    import torch
-
-    import int4_group_wise_b200 as q4
-    from int4_group_wise_b200 import inputs
-
-    if args.config not in (3, 4):
-        raise SystemExit("--variant stack runs config 3 or 4")
-    rank, world, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    peaks, peak_kind = load_peaks()
-    wl = inputs.workload(args.config)
-    gen = torch.Generator(device=dev).manual_seed(layer_seed(rank))
-    t0 = time.time()
-
-    def randn(shape, sigma):
-        return torch.randn(shape, generator=gen, device=dev, dtype=torch.float32).mul_(sigma)
-
-    X, H = {}, {}
-    for x_name, d in wl.calib.items():
-        x = torch.randn((wl.n_calib, d), generator=gen, device=dev, dtype=torch.float32)
-        cols = torch.randperm(d, generator=gen, device=dev)[:wl.outliers.get(x_name, 0)]
-        x[:, cols] *= 20.0
-        X[x_name] = x.to(torch.bfloat16)
-        del x
-        H[x_name] = torch.empty((d, d), dtype=torch.float32, device=dev)
-    ws = torch.empty(max([q4.hessian_workspace_bytes(wl.n_calib, d) for d in wl.calib.values()] + [16]),
-                     dtype=torch.uint8, device=dev)
-    alpha = torch.from_numpy(wl.alpha()).to(dev)
-    mats = []
-    for m in wl.matrices:
-        W = randn((m.d_out, m.d_in), wl.weight_sigma)
-        G = randn((m.d_out, m.d_in), 1e-3).to(torch.bfloat16)
-        # scales of matrices that are not searched: round-to-nearest (alpha = 1), fl(max|w_g| / 7)
-        delta = (W.abs().view(m.d_out, m.d_in // 32, 32).amax(-1) / 7.0).contiguous()
-        mats.append(dict(m=m, W=W, G=G, delta=delta, idx=torch.empty(delta.shape, dtype=torch.int32, device=dev),
-                         err=torch.empty_like(delta), Q=torch.empty_like(W), gW=torch.empty_like(W),
-                         gD=torch.empty_like(delta),
-                         packed=torch.empty((m.d_out, m.d_in // 2), dtype=torch.uint8, device=dev),
-                         scales=torch.empty(delta.shape, dtype=torch.float16, device=dev)))
-    gen_s = time.time() - t0
-    searched = [e for e in mats if e["m"].name in wl.searched]
-    n_weights = sum(e["W"].numel() for e in mats)
-    hess_flop = sum(float(wl.n_calib) * d * (d + 1) for d in wl.calib.values())
-    groups = sum(e["W"].numel() // 32 for e in searched)
-    K = int(alpha.numel())
-    stream = torch.cuda.current_stream(dev)
-    # independent matrices go round-robin to NS side streams (the small k/v launches alone leave
-    # most SMs idle); each stage starts after the previous one on every stream and ends when all
-    # side streams are done; each stream has its own Hessian workspace
-    NS = 4
-    side = [torch.cuda.Stream(device=dev) for _ in range(NS)]
-    wss = [ws] + [torch.empty_like(ws) for _ in range(NS - 1)]
-
-    def fan(launches):
-        go = torch.cuda.Event()
-        go.record(stream)
-        for s_ in side:
-            s_.wait_event(go)
-        for i, launch in enumerate(launches):
-            with torch.cuda.stream(side[i % NS]):
-                launch(i % NS)
-        for s_ in side:
-            done = torch.cuda.Event()
-            done.record(s_)
-            stream.wait_event(done)
-
-    def stage_hessian():
-        fan([lambda j, x=x_name: q4.hessian(X[x], H[x], wss[j]) for x_name in wl.calib])
-
-    def stage_search():
-        fan([lambda j, e=e: q4.scale_search(e["W"], H[e["m"].x_name], alpha, e["delta"], e["idx"], e["err"])
-             for e in searched])
-
-    def stage_lsq():
-        fan([lambda j, e=e: q4.lsq_fwd_bwd(e["W"], e["delta"], e["G"], q4.GRAD_SCALE, e["Q"], e["gW"], e["gD"])
-             for e in mats])
-
-    def stage_pack():
-        fan([lambda j, e=e: q4.pack_w4a16(e["W"], e["delta"], e["packed"], e["scales"]) for e in mats])
-
-    stages = [("hessian", stage_hessian), ("scale_search", stage_search), ("lsq_fwd_bwd", stage_lsq),
-              ("pack_w4a16", stage_pack)]
-
-    def step(ev=None):
-        for i, (_, fn) in enumerate(stages):
-            if ev is not None:
-                ev[i][0].record(stream)
-            fn()
-            if ev is not None:
-                ev[i][1].record(stream)
-
-    for _ in range(args.warmup):
-        step()
-    q4.sync_check()
-    evs = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in stages] for _ in range(args.steps)]
-    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    with ClockSampler(local, os.path.join(OUT_DIR, f"bench_stack_clocks_r{rank}.csv")) as clk:
-        start.record(stream)
-        for k in range(args.steps):
-            step(evs[k])
-        stop.record(stream)
-        torch.cuda.synchronize()
-    q4.sync_check()
-    total_ms = start.elapsed_time(stop) / args.steps
-    mean = {name: sum(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(args.steps)) / args.steps
-            for i, (name, _) in enumerate(stages)}
-    hbm = float(peaks["hbm_gbs"])
-    tc_peak = float(peaks["bf16_tflops"])
-    sm_max = float(peaks.get("sm_max_mhz", 1965.0))
-    search_roof = 148 * 128 * sm_max * 1e6 / (SEARCH_OPS_PER_CAND * K)
-    lsq_bytes = LSQ_BYTES_PER_ELT * n_weights
-    pack_bytes = PACK_BYTES_PER_ELT * n_weights
-    lsq_gbs = lsq_bytes / mean["lsq_fwd_bwd"] / 1e6
-    st = {
-        "hessian": {"value": hess_flop / mean["hessian"] / 1e9, "unit": "TFLOP/s", "ms": mean["hessian"],
-                    "launches": len(wl.calib), "flop": hess_flop,
-                    "frac": hess_flop / mean["hessian"] / 1e9 / tc_peak},
-        "scale_search": {"value": groups / mean["scale_search"] * 1e3, "unit": "groups/s",
-                         "ms": mean["scale_search"], "launches": len(searched), "groups": groups,
-                         "frac": groups / mean["scale_search"] * 1e3 / search_roof},
-        "lsq_fwd_bwd": {"value": lsq_gbs, "unit": "GB/s", "ms": mean["lsq_fwd_bwd"], "launches": len(mats),
-                        "bytes": lsq_bytes, "frac": lsq_gbs / hbm},
-        "pack_w4a16": {"value": pack_bytes / mean["pack_w4a16"] / 1e6, "unit": "GB/s", "ms": mean["pack_w4a16"],
-                       "launches": len(mats), "bytes": pack_bytes,
-                       "frac": pack_bytes / mean["pack_w4a16"] / 1e6 / hbm},
-    }
-    if rank == 0:
-        print(json.dumps({
-            "metric": METRIC, "value": lsq_gbs, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": total_ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "variant": "stack", "dtype": "f32", "data": "synthetic (drawn on the GPU)",
-            "config": {"workload": wl.title, "config_index": args.config, "matrices": len(mats),
-                       "weights": n_weights, "hessians": len(wl.calib), "n_calib": wl.n_calib,
-                       "searched_matrices": len(searched), "K": K,
-                       "streams": NS, "l2": "every stage's inputs are larger than L2; no flush"},
-            "stages": st, "peaks": {"hbm_gbs": hbm, "bf16_tflops": tc_peak, "kind": peak_kind,
-                                    "search_roof_groups_per_s": search_roof},
-            "gpu_launches": (len(wl.calib) * 2 + len(searched) + 2 * len(mats)) * args.steps,
-            "clocks": clk.summary(), "input_gen_s": round(gen_s, 1)}), flush=True)
 
 
 def run_per_channel(args):
@@ -631,7 +705,7 @@ def run_per_channel(args):
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
     peaks, peak_kind = load_peaks()
-    wl = inputs.workload(args.config)
+    wl = inputs.workload(1 if args.config is None else args.config)
     m = wl.matrices[0]
     W_h, G_h = wl.weight(m), wl.grad(m)
     R, C = W_h.shape
@@ -1051,26 +1125,35 @@ def run_refine(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--config", type=int, default=None, choices=[0, 1, 2, 3, 4],
+                    help="time only this workload as the headline (default: the 8B-class stack, then "
+                         "configs 1 and 2 under stages)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--variant", choices=["group32", "per-channel", "w4a16-decode", "fq-gemm", "hessian-split",
-                                          "refine", "stack"],
-                    default="group32",
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--variant", choices=["path", "per-channel", "w4a16-decode", "fq-gemm", "hessian-split",
+                                          "refine"],
+                    default="path",
                     help="per-channel: time the one-scale-per-row LSQ step and export instead; "
                          "w4a16-decode: time the inference GEMV on the packed 8B-class stack; "
                          "fq-gemm: time the fused fake-quant forward GEMM; "
                          "hessian-split: the calibration Hessian with its rows split over the ranks; "
-                         "refine: one sweep of the full-objective refinement; "
-                         "stack: the whole decoder stack of --config 3 or 4")
+                         "refine: one sweep of the full-objective refinement")
     ap.add_argument("--tokens", type=int, default=8192, help="fq-gemm: tokens of the micro-batch")
     ap.add_argument("--layers", type=int, default=None,
                     help="w4a16-decode: number of layers of the 8B-class stack (default: all 32)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if "WORLD_SIZE" not in os.environ:
+        if args.gpus > 1:          # one process per GPU: start the ranks, then report their status
+            sys.exit(relaunch_ranks(args.gpus, sys.argv[1:]))
+    elif int(os.environ["WORLD_SIZE"]) != args.gpus:
+        ap.error(f"--gpus {args.gpus} but the launcher started WORLD_SIZE={os.environ['WORLD_SIZE']} ranks")
     if args.impl == "reference":
         run_reference(args)
     elif args.variant == "per-channel":
@@ -1083,8 +1166,6 @@ def main():
         run_hessian_split(args)
     elif args.variant == "refine":
         run_refine(args)
-    elif args.variant == "stack":
-        run_stack(args)
     else:
         run_ours(args)
 

@@ -49,3 +49,16 @@ def test_workload_shapes():
     w0 = inputs.workload(0)
     assert w0.g_dtype == "f32" and w0.K == 101 and w0.matrices[0].d_in == 512
     assert inputs.workload(2).K == 201
+
+
+def test_row_prefix_has_the_full_tensors_bytes():
+    """weight(rows=r) / grad(rows=r) / activations(n=r) are the first r rows of the full tensors
+    (the bounded CPU samples of the benchmark rely on it)."""
+    w2 = inputs.workload(2)
+    m2 = w2.matrices[0]
+    full = w2.weight(m2)
+    np.testing.assert_array_equal(w2.weight(m2, rows=100), full[:100])
+    np.testing.assert_array_equal(w2.grad(m2, rows=64), w2.grad(m2)[:64])
+    w0 = inputs.workload(0)
+    np.testing.assert_array_equal(w0.activations("x", n=300), w0.activations("x")[:300])
+    np.testing.assert_array_equal(w0.weight(w0.matrices[0], rows=17), w0.weight(w0.matrices[0])[:17])

@@ -55,12 +55,30 @@ def test_single_process_aggregation_is_identity():
     assert bench.aggregate_over_ranks(5.0, 1.5) == (5.0, 1.5)
 
 
-def test_reference_arm_prints_only_on_rank0(tmp_path):
-    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
-    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+def test_gpus_flag_launches_that_many_ranks():
+    """`bench.py --gpus 2` without a launcher re-executes itself under torch.distributed.run with
+    two ranks (gloo on CPU for the reference arm): exactly one JSON line, from rank 0, reporting
+    both ranks; the other rank exits 0 without work."""
+    import json
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+                        "--config", "0", "--steps", "1", "--warmup", "3"], env=env, capture_output=True,
+                       text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["n_gpus"] == 2
+    assert set(rec["stages"]) == {"hessian_gflops", "scale_search_groups_per_s", "lsq_fwd_bwd_gbs",
+                                  "pack_w4a16_gbs"}
+
+
+def test_gpus_flag_must_match_the_launchers_world_size():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="2", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "4", "--impl", "reference",
                         "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True,
                        timeout=300, cwd=ROOT)
-    assert r.returncode == 0 and r.stdout.strip() == ""
+    assert r.returncode != 0 and "WORLD_SIZE=2" in r.stderr
 
 
 # ------------------------------------------------------------- split-n Hessian plumbing
