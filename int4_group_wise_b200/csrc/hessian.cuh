@@ -18,14 +18,18 @@
 // are loaded once.  No load is multicast.
 //
 // Warps of each CTA:
-//   warp 0      TMA producer: 64-row x 64-column boxes of X, 128-byte
-//               swizzle, into a 6-stage ring; the peer CTA's copies complete
-//               on the leader's full barrier, which the leader arms with the
-//               bytes of both CTAs;
+//   warp 0      TMA producer: 128-row x 64-column boxes of X, 128-byte
+//               swizzle, into a 3-stage ring of 128-row stages; the peer
+//               CTA's copies complete on the leader's full barrier, which the
+//               leader arms with the bytes of both CTAs;
 //   warp 1      allocates the pair's 512 TMEM columns; in the leader CTA one
 //               thread issues the MMAs; each commit frees the ring slot in
 //               both CTAs;
 //   warps 2..5  epilogue over TMEM lanes 32*(w%4)..+31 (= the CTA's rows).
+// A stage holds 128 rows of X: eight K = 16 MMAs per stage between two
+// barrier hand-offs.  (With 64-row stages, four MMAs per wait-and-commit, the
+// tensor pipe idled about a quarter of its cycles at the stage boundaries; at
+// 128 rows it runs at the rate of MMAs issued with no hand-off at all.)
 // Chunked promotion: the tensor core accumulates kPChunkKB stages (16384 rows)
 // into TMEM columns [0,256); the epilogue adds each finished chunk into a
 // float32 master copy in columns [256,512) with IEEE round-to-nearest adds
@@ -50,14 +54,14 @@ namespace qat4 {
 
 constexpr int kPTile = 256;                   // tile rows = tile columns
 constexpr int kPHalf = 128;                   // rows (A) / columns (B) held by one CTA
-constexpr int kPBK = 64;                      // X rows per pipeline stage
-constexpr int kPStages = 6;
+constexpr int kPBK = 128;                     // X rows per pipeline stage
+constexpr int kPStages = 3;
 constexpr int kPThreads = 192;
-constexpr int kPChunkKB = 256;                // stages per promotion chunk (16384 rows)
+constexpr int kPChunkKB = 128;                // stages per promotion chunk (16384 rows)
 constexpr int kPPairsPerGpu = 74;             // SM pairs of a B200; fixes the split of n
-constexpr uint32_t kPBoxBytes = 64 * kPBK * 2;          // one 64x64 bf16 box = 8 KB
-constexpr uint32_t kPOperandBytes = 2 * kPBoxBytes;     // 128 columns = 16 KB
-constexpr uint32_t kPStageBytes = 2 * kPOperandBytes;   // A half + B half = 32 KB
+constexpr uint32_t kPBoxBytes = 64 * kPBK * 2;          // one 64-column x 128-row bf16 box = 16 KB
+constexpr uint32_t kPOperandBytes = 2 * kPBoxBytes;     // 128 columns = 32 KB
+constexpr uint32_t kPStageBytes = 2 * kPOperandBytes;   // A half + B half = 64 KB
 constexpr uint32_t kPSmemBytes = kPStages * kPStageBytes + 1024;
 constexpr uint32_t kPTmemCols = 512;                    // [0,256) accumulator, [256,512) master
 
@@ -72,8 +76,8 @@ constexpr uint32_t kPIdesc = (1u << 4)            // D format: F32
                            | ((256u >> 4) << 24); // M >> 4
 
 // Shared-memory matrix descriptor for one 128-column operand half laid out as
-// [2 column blocks of 64][64 rows][128 B], 128-byte swizzle: leading byte
-// offset = distance between the two 64-column blocks (8 KB), stride byte
+// [2 column blocks of 64][128 rows][128 B], 128-byte swizzle: leading byte
+// offset = distance between the two 64-column blocks (16 KB), stride byte
 // offset = distance between 8-row groups (1 KB).
 __device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr) {
     uint64_t d = 0;
@@ -97,7 +101,7 @@ __host__ __device__ __forceinline__ void hess_tile_coords(int t, int nb, int& I,
 struct HessPlan {
     int nb;        // ceil(C / 256)
     int tiles;     // nb (nb + 1) / 2
-    int kblocks;   // ceil(n / 64)
+    int kblocks;   // ceil(n / 128): pipeline stages over the calibration rows
     int split;     // S
 };
 

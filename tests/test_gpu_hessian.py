@@ -88,7 +88,7 @@ def test_hessian_full_size_every_tile(cfg, cache, oracle_mod):
 @pytest.mark.parametrize("n,C", [(40000, 3072), (50000, 2048), (20000, 512)])
 def test_hessian_multi_chunk_ragged(n, C, oracle_mod):
     """n spans several 16384-row promotion chunks with a ragged last chunk and a ragged last
-    64-row stage; (40000, 3072) stores H directly, the others split n and reduce partials."""
+    128-row stage; (40000, 3072) stores H directly, the others split n and reduce partials."""
     Xb = inputs.activations(n, C, seed=n, cfg=62, name="X", outliers=C // 100)
     X, H = _gpu_h(Xb)
     Hg = H.cpu().numpy()
