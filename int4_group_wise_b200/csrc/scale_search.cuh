@@ -25,6 +25,14 @@
 // without overflow; scaling by powers of two leaves the codes and the argmin
 // unchanged.
 //
+// Equilibration: when the binary16 split of the block would lose too much
+// (its split-error ratio kappa_d above 2^-17 -- channels whose scales differ
+// by a few hundred put the small entries below binary16's normal range, and
+// every candidate of such a block would then be re-scored), the block is
+// first scaled to H' = D^-1 H D^-1 with d_i a power of two near sqrt|H_ii|,
+// and the error vectors to e' = D e, so that e' H' e' = e H e exactly; the
+// bound below is then taken for (H', e').
+//
 // Two-stage pipeline: while the tensor core multiplies candidate k, the
 // threads quantize candidate k + 1.  Each thread parks its v of a candidate in
 // TMEM next to that candidate's P (columns 64s..64s+31 hold P of stage s,
@@ -55,6 +63,11 @@
 namespace qat4 {
 
 constexpr int kTri = 528;          // entries of the upper triangle of a 32x32 block
+
+template <bool B>
+struct BoolTag {
+    static constexpr bool value = B;
+};
 constexpr float kMagic = 12582912.0f;          // 1.5 * 2^23: x + M - M = rint(x) for |x| < 2^22
 constexpr float kTieWindow = 0.5f - 3.814697265625e-06f;  // 0.5 - 2^-18
 
@@ -105,8 +118,11 @@ struct SearchTcSmem {
     int exact_block;              // the split cannot represent this block: re-score every candidate
     int abort;
     float coef, coef_f, tsum;
-    alignas(16) float sd[32];     // sqrt(sigma_H |H_ii|), rounded up
+    alignas(16) float sd[32];     // sqrt(sigma_H |H'_ii|), rounded up
     float isd[32];                // reciprocals rounded up (set-up only)
+    alignas(16) float dsc[32];    // equilibration d_i (powers of two; all 1 unless equilibrated)
+    float idsc[32];               // 1 / d_i
+    int eq;                       // the block is equilibrated: H' = D^-1 H D^-1, e' = D e
 };
 constexpr size_t kTcSmemBytes = sizeof(SearchTcSmem) + 1024;   // + alignment of the operand tiles
 static_assert(offsetof(SearchTcSmem, a) == 0 && offsetof(SearchTcSmem, bhi) % 1024 == 0 &&
@@ -137,13 +153,14 @@ __device__ __noinline__ void tc_error_exact(const float* __restrict__ wrow, floa
 // Start of row i of the row-major upper triangle (j >= i) of a 32x32 matrix.
 __host__ __device__ constexpr int tri_start(int i) { return 32 * i - (i * (i - 1)) / 2; }
 
-// float64 value of one candidate (the re-score): the exact codes (w * (1/dk),
+// float64 value of one candidate (the re-score; out of line, so that its 32 binary64
+// differences do not add to the candidate loop's registers): the exact codes (w * (1/dk),
 // with the IEEE division redone for the group near a rounding boundary or when
 // 1/dk is not finite, as in the screen), Q = fl(dk * q), the exact difference
 // e = w - Q (exact in binary64), and e H' e summed in binary64 over the upper
 // triangle H' (H'_ij = H_ij + H_ji, H'_ii = H_ii).  Four rows at a time, each
 // row's sum split in two, so eight independent FMA chains are in flight.
-__device__ __forceinline__ double tc_quad_form64(const double* h64, const float (&w)[32], float dk) {
+__device__ __noinline__ double tc_quad_form64(const double* h64, const float (&w)[32], float dk) {
     double ed[32];
     const float rc = __frcp_rn(dk);
     float fmax_abs = 0.0f;
@@ -179,9 +196,12 @@ __device__ __forceinline__ double tc_quad_form64(const double* h64, const float 
 
 // Quantizes one candidate for this thread's row: writes e_hi into the stage's
 // half of its A row, parks v = 2e - e_hi in the stage's TMEM columns (this
-// thread's lane) and returns S = sum |v_i| sd_i.
+// thread's lane) and returns S = sum |v_i| sd_i.  For an equilibrated block e
+// is first scaled to D e.
+template <bool EQ>
 __device__ __forceinline__ float tc_quantize(const float2 (&ws)[16], float dk, float sig, bool screen,
                                              const float* __restrict__ wrow, float* eslot, const float* sd,
+                                             const float* dsc,
                                              uint32_t a_row, uint32_t swz, uint32_t stage, uint32_t tv) {
     const float ds = __fmul_rn(dk, sig);                              // scaled (exact power of two)
     const float rc = __frcp_rn(ds);
@@ -211,6 +231,15 @@ __device__ __forceinline__ float tc_quantize(const float2 (&ws)[16], float dk, f
             const float4 x = e4[c];
             v[2 * c] = make_float2(x.x, x.y);
             v[2 * c + 1] = make_float2(x.z, x.w);
+        }
+    }
+    if (EQ) {            // equilibrated block: e' = D e (powers of two, exact)
+        const float4* d4 = reinterpret_cast<const float4*>(dsc);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float4 dd = d4[c];
+            v[2 * c] = __fmul2_rn(v[2 * c], make_float2(dd.x, dd.y));
+            v[2 * c + 1] = __fmul2_rn(v[2 * c + 1], make_float2(dd.z, dd.w));
         }
     }
     const float2 two = make_float2(2.0f, 2.0f);
@@ -337,87 +366,131 @@ scale_search_kernel(const float* __restrict__ W, int R, int C,
         reinterpret_cast<uint4*>(sm.bhi)[x] = make_uint4(0u, 0u, 0u, 0u);    // bhi and blo are contiguous
     __syncthreads();
 
-    // 1/sqrt|H_ii| rounded up (for kappa): an upper bound of the true reciprocal
-    if (tid < 32) sm.isd[tid] = __fdiv_ru(1.0f, __fsqrt_rd(fabsf(sm.u.hfull[tid][tid])));
-    __syncthreads();
-
-    // H' for the float64 re-score, kappa, and the largest |(H_ij + H_ji)/2|
-    float kap = 0.0f, hmax = 0.0f;
+    // float64 table of the block for the re-score: H'_ij = H_ij + H_ji (j > i), H'_ii = H_ii (unscaled)
     for (int x = tid; x < 32 * 32; x += kTcRows) {
         const int i = x >> 5, j = x & 31;
-        const float a = sm.u.hfull[i][j], b = sm.u.hfull[j][i];
-        const float hs = up(fabs(0.5 * (static_cast<double>(a) + static_cast<double>(b))));
-        hmax = fmaxf(hmax, (hs <= 3.4028234663852886e38f) ? hs : __int_as_float(0x7f800000));
-        if (j == i) {
-            sm.h64[tri_start(i)] = static_cast<double>(a);
-        } else if (j > i) {
-            sm.h64[tri_start(i) + (j - i)] = static_cast<double>(a) + static_cast<double>(b);
-            const float m = fmaxf(fabsf(a), fabsf(b));
-            if (m != 0.0f) {
-                const float ratio = __fmul_ru(__fmul_ru(m, sm.isd[i]), sm.isd[j]);
-                kap = fmaxf(kap, (ratio <= 3.4028234663852886e38f) ? ratio : __int_as_float(0x7f800000));
+        if (j == i)
+            sm.h64[tri_start(i)] = static_cast<double>(sm.u.hfull[i][j]);
+        else if (j > i)
+            sm.h64[tri_start(i) + (j - i)] =
+                static_cast<double>(sm.u.hfull[i][j]) + static_cast<double>(sm.u.hfull[j][i]);
+    }
+    // The binary16 split and its bound, first for the block as it is (pass 0), then -- only if
+    // that split's error ratio kappa_d exceeds 2^-17 -- for the equilibrated block
+    // D^-1 H D^-1 (pass 1).  Every quantity below is of the block of the pass: entries
+    // a' = a / (d_i d_j), exact in binary64 since the d_i are powers of two.
+    for (int pass = 0; pass < 2; ++pass) {
+        if (tid < 32) {
+            float d = 1.0f;
+            if (pass == 1) {   // a power of two near sqrt|H_ii|: H_ii / d^2 in [1, 4)
+                const float h = fabsf(sm.u.hfull[tid][tid]);
+                if (h >= 1.1754943508222875e-38f && h <= 3.4028234663852886e38f) {
+                    const int e = static_cast<int>((__float_as_uint(h) >> 23) & 0xFF) - 127;
+                    d = __uint_as_float(static_cast<uint32_t>(127 + (e >> 1)) << 23);
+                }
+            }
+            sm.dsc[tid] = d;
+            sm.idsc[tid] = 1.0f / d;     // exact: d is a power of two
+        }
+        if (tid == 0) {
+            sm.kappa_bits = __float_as_uint(1.0f);
+            sm.kappa_d_bits = 0u;
+            sm.hmax_bits = 0u;
+            sm.eq = pass;
+        }
+        __syncthreads();
+
+        // 1/sqrt|H'_ii| rounded up (for kappa): an upper bound of the true reciprocal
+        if (tid < 32) {
+            const double hd = static_cast<double>(sm.u.hfull[tid][tid]) *
+                              (static_cast<double>(sm.idsc[tid]) * static_cast<double>(sm.idsc[tid]));
+            sm.isd[tid] = __fdiv_ru(1.0f, __fsqrt_rd(__double2float_rd(fabs(hd))));
+        }
+        __syncthreads();
+
+        // kappa and the largest |(H'_ij + H'_ji)/2|
+        float kap = 0.0f, hmax = 0.0f;
+        for (int x = tid; x < 32 * 32; x += kTcRows) {
+            const int i = x >> 5, j = x & 31;
+            const double dij = static_cast<double>(sm.idsc[i]) * static_cast<double>(sm.idsc[j]);   // exact
+            const double a = static_cast<double>(sm.u.hfull[i][j]) * dij, b = static_cast<double>(sm.u.hfull[j][i]) * dij;
+            const float hs = up(fabs(0.5 * (a + b)));
+            hmax = fmaxf(hmax, (hs <= 3.4028234663852886e38f) ? hs : __int_as_float(0x7f800000));
+            if (j > i) {
+                const float mm = up(fmax(fabs(a), fabs(b)));
+                if (mm != 0.0f) {
+                    const float ratio = __fmul_ru(__fmul_ru(mm, sm.isd[i]), sm.isd[j]);
+                    kap = fmaxf(kap, (ratio <= 3.4028234663852886e38f) ? ratio : __int_as_float(0x7f800000));
+                }
             }
         }
-    }
-    {   // non-negative floats order like their bit patterns: one shared atomic per warp
-        const unsigned kb = __reduce_max_sync(0xffffffffu, __float_as_uint(kap));
-        const unsigned hb = __reduce_max_sync(0xffffffffu, __float_as_uint(hmax));
-        if ((tid & 31) == 0) {
-            atomicMax(&sm.kappa_bits, kb);
-            atomicMax(&sm.hmax_bits, hb);
+        {   // non-negative floats order like their bit patterns: one shared atomic per warp
+            const unsigned kb = __reduce_max_sync(0xffffffffu, __float_as_uint(kap));
+            const unsigned hb = __reduce_max_sync(0xffffffffu, __float_as_uint(hmax));
+            if ((tid & 31) == 0) {
+                atomicMax(&sm.kappa_bits, kb);
+                atomicMax(&sm.hmax_bits, hb);
+            }
         }
-    }
-    __syncthreads();
+        __syncthreads();
 
-    // scale of the block: 2^13 <= hmax * sigma_H < 2^14
-    const float hmx = __uint_as_float(sm.hmax_bits);
-    const bool hbad = !(hmx >= 1.0e-30f) || !(hmx <= 1.0e30f);
-    const int eh = hbad ? 0 : static_cast<int>((__float_as_uint(hmx) >> 23) & 0xFF) - 127;
-    const float sigH = __uint_as_float(static_cast<uint32_t>(127 + 13 - eh) << 23);
-    if (tid < 32) {
-        const float sd = hbad ? 0.0f : __fsqrt_ru(__fmul_ru(fabsf(sm.u.hfull[tid][tid]), sigH));
-        sm.sd[tid] = sd;
-        sm.isd[tid] = __fdiv_ru(1.0f, sd);          // for kappa_d (inf when sd = 0)
-    }
-    __syncthreads();
-
-    // binary16 split of the scaled symmetrised block; entry (k, n) goes to row n, column k of B
-    float kapd = 0.0f;
-    for (int x = tid; x < 32 * 32; x += kTcRows) {
-        const int k = x >> 5, n = x & 31;
-        const double s = 0.5 * (static_cast<double>(sm.u.hfull[k][n]) + static_cast<double>(sm.u.hfull[n][k])) *
-                         static_cast<double>(sigH);
-        __half hi = __float2half_rn(static_cast<float>(s));
-        if (!(fabsf(__half2float(hi)) >= 6.103515625e-05f)) hi = __float2half_rn(0.0f);   // no subnormal parts
-        const double r1 = s - static_cast<double>(__half2float(hi));
-        __half lo = __float2half_rn(static_cast<float>(r1));
-        if (!(fabsf(__half2float(lo)) >= 6.103515625e-05f)) lo = __float2half_rn(0.0f);
-        const float dlt = up(fabs(r1 - static_cast<double>(__half2float(lo))));
-        if (dlt != 0.0f) {
-            const float ratio = __fmul_ru(__fmul_ru(dlt, sm.isd[k]), sm.isd[n]);
-            kapd = fmaxf(kapd, (ratio <= 3.4028234663852886e38f) ? ratio : __int_as_float(0x7f800000));
+        // scale of the block: 2^13 <= hmax * sigma_H < 2^14
+        const float hmx = __uint_as_float(sm.hmax_bits);
+        const bool hbad = !(hmx >= 1.0e-30f) || !(hmx <= 1.0e30f);
+        const int eh = hbad ? 0 : static_cast<int>((__float_as_uint(hmx) >> 23) & 0xFF) - 127;
+        const double sigH = static_cast<double>(__uint_as_float(static_cast<uint32_t>(127 + 13 - eh) << 23));
+        if (tid < 32) {
+            const double hd = static_cast<double>(sm.u.hfull[tid][tid]) *
+                              (static_cast<double>(sm.idsc[tid]) * static_cast<double>(sm.idsc[tid]));
+            const float sd = hbad ? 0.0f : __fsqrt_ru(up(fabs(hd) * sigH));
+            sm.sd[tid] = sd;
+            sm.isd[tid] = __fdiv_ru(1.0f, sd);          // for kappa_d (inf when sd = 0)
         }
-        const uint32_t off = sw128_off(static_cast<uint32_t>(n), static_cast<uint32_t>(k >> 3)) + (k & 7) * 2;
-        *reinterpret_cast<__half*>(sm.bhi + off) = hi;
-        *reinterpret_cast<__half*>(sm.blo + off) = lo;
-    }
-    {
-        const unsigned db = __reduce_max_sync(0xffffffffu, __float_as_uint(kapd));
-        if ((tid & 31) == 0) atomicMax(&sm.kappa_d_bits, db);
-    }
-    __syncthreads();
-    if (tid == 0) {
-        const double kp = static_cast<double>(__uint_as_float(sm.kappa_bits));
-        const double kd = static_cast<double>(__uint_as_float(sm.kappa_d_bits));
-        double ts = 0.0;
-        for (int i = 0; i < 32; ++i) ts += static_cast<double>(sm.sd[i]);
-        const double tau = 7.62939453125e-06;                         // 2^-17
-        const double c = (kp + kd) * (tau + 1.9073486328125e-06 + 2.384185791015625e-07) + kd +
-                         kp * (9.5367431640625e-07 + 1.1920928955078125e-07);
-        sm.coef = up(c * 1.02);
-        sm.coef_f = up((kp + kd) * 2.44140625e-04 * 1.02);            // 2^-12
-        sm.tsum = up(ts * (1.0 + 1e-6));
-        sm.exact_block = (hbad || !(sm.coef <= 1.0e30f) || !(sm.coef_f <= 1.0e30f)) ? 1 : 0;
+        __syncthreads();
+
+        // binary16 split of the scaled symmetrised block; entry (k, n) goes to row n, column k of B
+        float kapd = 0.0f;
+        for (int x = tid; x < 32 * 32; x += kTcRows) {
+            const int k = x >> 5, n = x & 31;
+            const double dkn = static_cast<double>(sm.idsc[k]) * static_cast<double>(sm.idsc[n]);   // exact
+            const double s = 0.5 * (static_cast<double>(sm.u.hfull[k][n]) + static_cast<double>(sm.u.hfull[n][k])) *
+                             dkn * sigH;
+            __half hi = __float2half_rn(static_cast<float>(s));
+            if (!(fabsf(__half2float(hi)) >= 6.103515625e-05f)) hi = __float2half_rn(0.0f);   // no subnormal parts
+            const double r1 = s - static_cast<double>(__half2float(hi));
+            __half lo = __float2half_rn(static_cast<float>(r1));
+            if (!(fabsf(__half2float(lo)) >= 6.103515625e-05f)) lo = __float2half_rn(0.0f);
+            const float dlt = up(fabs(r1 - static_cast<double>(__half2float(lo))));
+            if (dlt != 0.0f) {
+                const float ratio = __fmul_ru(__fmul_ru(dlt, sm.isd[k]), sm.isd[n]);
+                kapd = fmaxf(kapd, (ratio <= 3.4028234663852886e38f) ? ratio : __int_as_float(0x7f800000));
+            }
+            const uint32_t off = sw128_off(static_cast<uint32_t>(n), static_cast<uint32_t>(k >> 3)) + (k & 7) * 2;
+            *reinterpret_cast<__half*>(sm.bhi + off) = hi;
+            *reinterpret_cast<__half*>(sm.blo + off) = lo;
+        }
+        {
+            const unsigned db = __reduce_max_sync(0xffffffffu, __float_as_uint(kapd));
+            if ((tid & 31) == 0) atomicMax(&sm.kappa_d_bits, db);
+        }
+        __syncthreads();
+        if (tid == 0) {
+            const double kp = static_cast<double>(__uint_as_float(sm.kappa_bits));
+            const double kd = static_cast<double>(__uint_as_float(sm.kappa_d_bits));
+            double ts = 0.0;
+            for (int i = 0; i < 32; ++i) ts += static_cast<double>(sm.sd[i]);
+            const double tau = 7.62939453125e-06;                         // 2^-17
+            const double c = (kp + kd) * (tau + 1.9073486328125e-06 + 2.384185791015625e-07) + kd +
+                             kp * (9.5367431640625e-07 + 1.1920928955078125e-07);
+            sm.coef = up(c * 1.02);
+            sm.coef_f = up((kp + kd) * 2.44140625e-04 * 1.02);            // 2^-12
+            sm.tsum = up(ts * (1.0 + 1e-6));
+            sm.exact_block = (hbad || !(sm.coef <= 1.0e30f) || !(sm.coef_f <= 1.0e30f)) ? 1 : 0;
+        }
+        __syncthreads();
+        // keep this pass unless its split is poor and the block can be equilibrated
+        if (pass == 1 || hbad || !(__uint_as_float(sm.kappa_d_bits) > 7.62939453125e-06f)) break;
+        __syncthreads();
     }
     fence_proxy_async_smem();
     __syncthreads();
@@ -448,9 +521,23 @@ scale_search_kernel(const float* __restrict__ W, int R, int C,
     for (int j = 0; j < 16; ++j) m = fmaxf(m, fmaxf(fabsf(ws[j].x), fabsf(ws[j].y)));
     const bool zero = (m == 0.0f);
     const float base = __fdiv_rn(m, 7.0f);
+    const bool eq = sm.eq != 0;
+    float md = m;        // the largest |w_i| d_i: m unless the block is equilibrated
+    if (eq) {
+        md = 0.0f;
+        const float4* d4 = reinterpret_cast<const float4*>(sm.dsc);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            const float4 dd = d4[c];
+            md = fmaxf(md, fmaxf(fabsf(ws[2 * c].x) * dd.x, fabsf(ws[2 * c].y) * dd.y));
+            md = fmaxf(md, fmaxf(fabsf(ws[2 * c + 1].x) * dd.z, fabsf(ws[2 * c + 1].y) * dd.w));
+        }
+    }
     // exact_row: the power-of-two row scale would leave binary32 range; re-score every candidate
-    const bool exact_row = exact_block || !(m >= 7.888609052210118e-31f);      // 2^-100
-    const int em = exact_row ? 0 : static_cast<int>((__float_as_uint(m) >> 23) & 0xFF) - 127;
+    const bool exact_row = exact_block || !(m >= 7.888609052210118e-31f) ||      // 2^-100
+                           !(md >= 7.888609052210118e-31f) || !(md <= 1.2676506002282294e30f);   // 2^100
+    // row scale: 2^13 <= max_i |w_i| d_i sigma < 2^14, so every |e_i d_i| sigma < 2^14
+    const int em = exact_row ? 0 : static_cast<int>((__float_as_uint(md) >> 23) & 0xFF) - 127;
     const float sig = __uint_as_float(static_cast<uint32_t>(127 + 13 - em) << 23);
     const bool screen = valid && !zero && !exact_row;
 #pragma unroll
@@ -469,41 +556,47 @@ scale_search_kernel(const float* __restrict__ W, int R, int C,
     float upper = __int_as_float(0x7f800000);
     bool ok = true;
 
-    // prologue: candidate 0 into stage 0
-    float S0 = tc_quantize(ws, __fmul_rn(__ldg(alpha), base), sig, screen, wrow, eslot, sm.sd, a_row, swz, 0u,
-                           tlane + 32u);
-    float S1 = 0.0f;
-    tmem_st_wait();
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) tc_issue(tmem, a0, bh, bl, &sm.mbar[0]);
+    float S0 = 0.0f, S1 = 0.0f;
+    // the candidate loop, compiled once for plain and once for equilibrated blocks
+    auto candidate_loop = [&](auto eq_tag) {
+        constexpr bool EQ = decltype(eq_tag)::value;
+        // prologue: candidate 0 into stage 0
+        S0 = tc_quantize<EQ>(ws, __fmul_rn(__ldg(alpha), base), sig, screen, wrow, eslot, sm.sd, sm.dsc, a_row,
+                             swz, 0u, tlane + 32u);
+        tmem_st_wait();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) tc_issue(tmem, a0, bh, bl, &sm.mbar[0]);
 
-    // steady state, two candidates per trip so the stages alternate statically: quantize
-    // candidate k + 1 into the other stage, hand it to the tensor core, then consume k
-    for (int k = 0; k < K; k += 2) {
-        if (k + 1 < K) {
-            S1 = tc_quantize(ws, __fmul_rn(__ldg(alpha + k + 1), base), sig, screen, wrow, eslot, sm.sd, a_row, swz,
-                             1u, tlane + kTcStageCols + 32u);
-            tmem_st_wait();
-            fence_proxy_async_smem();
-            tc_fence_before();
-            if (__syncthreads_or(!ok)) { ok = false; break; }
-            if (lane0 && warp == ((k + 1) & 3)) tc_issue(tmem + kTcStageCols, a0 + 64u, bh, bl, &sm.mbar[1]);
+        // steady state, two candidates per trip so the stages alternate statically: quantize
+        // candidate k + 1 into the other stage, hand it to the tensor core, then consume k
+        for (int k = 0; k < K; k += 2) {
+            if (k + 1 < K) {
+                S1 = tc_quantize<EQ>(ws, __fmul_rn(__ldg(alpha + k + 1), base), sig, screen, wrow, eslot, sm.sd,
+                                     sm.dsc, a_row, swz, 1u, tlane + kTcStageCols + 32u);
+                tmem_st_wait();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                if (__syncthreads_or(!ok)) { ok = false; break; }
+                if (lane0 && warp == ((k + 1) & 3)) tc_issue(tmem + kTcStageCols, a0 + 64u, bh, bl, &sm.mbar[1]);
+            }
+            if (ok) ok = tc_consume(k, tlane, &sm.mbar[0], &sm.abort, limit_ns, S0, tb, top, upper);
+            if (k + 1 >= K) break;
+            if (k + 2 < K) {
+                S0 = tc_quantize<EQ>(ws, __fmul_rn(__ldg(alpha + k + 2), base), sig, screen, wrow, eslot, sm.sd,
+                                     sm.dsc, a_row, swz, 0u, tlane + 32u);
+                tmem_st_wait();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                if (__syncthreads_or(!ok)) { ok = false; break; }
+                if (lane0 && warp == ((k + 2) & 3)) tc_issue(tmem, a0, bh, bl, &sm.mbar[0]);
+            }
+            if (ok) ok = tc_consume(k + 1, tlane + kTcStageCols, &sm.mbar[1], &sm.abort, limit_ns, S1, tb, top, upper);
         }
-        if (ok) ok = tc_consume(k, tlane, &sm.mbar[0], &sm.abort, limit_ns, S0, tb, top, upper);
-        if (k + 1 >= K) break;
-        if (k + 2 < K) {
-            S0 = tc_quantize(ws, __fmul_rn(__ldg(alpha + k + 2), base), sig, screen, wrow, eslot, sm.sd, a_row, swz,
-                             0u, tlane + 32u);
-            tmem_st_wait();
-            fence_proxy_async_smem();
-            tc_fence_before();
-            if (__syncthreads_or(!ok)) { ok = false; break; }
-            if (lane0 && warp == ((k + 2) & 3)) tc_issue(tmem, a0, bh, bl, &sm.mbar[0]);
-        }
-        if (ok) ok = tc_consume(k + 1, tlane + kTcStageCols, &sm.mbar[1], &sm.abort, limit_ns, S1, tb, top, upper);
-    }
+    };
+    if (eq) candidate_loop(BoolTag<true>{});
+    else candidate_loop(BoolTag<false>{});
     tc_fence_before();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, kTcTmemCols);

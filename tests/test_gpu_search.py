@@ -155,3 +155,23 @@ def test_search_degenerate_blocks_rows_and_ties(oracle_mod):
     torch.cuda.synchronize()
     assert torch.all(i2 % 3 == 0)                                     # first of each equal triple
     check_search(W, H, rep, oracle_mod)
+
+
+@pytest.mark.parametrize("spread,seed", [(8, 11), (14, 12), (20, 13)])
+def test_search_widely_scaled_channels(spread, seed, oracle_mod):
+    """Channel scales spread over 2^-spread/2 .. 2^spread/2 (and lognormal channels with a strongly
+    correlated pair): the binary16 split of such blocks puts the small entries below binary16's
+    normal range, so the kernel equilibrates them (H' = D^-1 H D^-1, e' = D e) before the screen.
+    Every row and group against the oracle."""
+    rng = np.random.default_rng(seed)
+    R, C, n = 200, 128, 4096
+    X = rng.standard_normal((n, C)).astype(f32)
+    X *= (2.0 ** rng.uniform(-spread / 2, spread / 2, C)).astype(f32)
+    X[:, 5] = X[:, 4] * f32(1e-3) + X[:, 5] * f32(1e-6)      # nearly collinear pair, very different scales
+    Xb = inputs.f32_to_bf16_bits(X)
+    H = _hessian_fp32(oracle_mod, Xb)
+    W = inputs.gaussian((R, C), 0.02, seed=seed, cfg=51, name="W")
+    W[1] *= f32(1e-20)                                          # tiny rows
+    W[2, :32] = f32(0.02) * np.sign(W[2, :32])                 # equal magnitudes
+    alpha = inputs.alpha_grid(0.3, 0.0035, 201)
+    check_search(W, H, alpha, oracle_mod)
