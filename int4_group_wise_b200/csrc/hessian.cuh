@@ -36,12 +36,20 @@
 // (the tensor core's own accumulation over 262144 rows drifts by more than
 // 1e-3), then releases the accumulator to the MMA.
 //
-// Split of n: with T upper tiles, each tile's n range is cut into S equal
-// parts, S = max(1, min(74 / T, kblocks / 16)) -- a function of (n, C) only,
-// so the result does not depend on the device.  With S = 1 the epilogue
-// scales by 1/n and stores H directly; with S > 1 it stores its fp32 partial
-// into the workspace and hessian_reduce_kernel adds the S partials of every
-// tile in fixed order, scales and stores H -- deterministic.
+// Split of n: a unit is one CTA pair computing one tile over a part of the
+// calibration rows.  With T <= 74 upper tiles, every tile's rows are cut into
+// S = max(1, min(74 / T, kblocks / 16)) equal parts.  With more tiles, the
+// tiles run one per unit in waves of 74 pairs; when the last wave would be
+// partly empty (r = T mod 74 tiles), those r tiles -- the last ones, launched
+// last -- are cut into S_t = min(74 / r, kblocks / 16) parts so that the last
+// wave is full and 1/S_t as long (C = 8192: 528 tiles, 7.14 waves instead of
+// 8).  Units with the same part index walk the same calibration rows at the
+// same time, so X stays shared through L2.  The plan is a function of (n, C)
+// only, so the result does not depend on the device.  A tile in one part is
+// scaled by 1/n and stored with its mirror directly; a tile in several parts
+// stores its fp32 partials into the workspace (at most 74 of them) and
+// hessian_reduce_kernel adds them in fixed order, scales and stores the tile
+// -- deterministic.
 //
 // Every mbarrier wait is bounded (device_common.cuh); on a timeout a CTA stops
 // issuing work, waits (bounded) for its own copies and MMAs in flight, frees
@@ -100,9 +108,11 @@ __host__ __device__ __forceinline__ void hess_tile_coords(int t, int nb, int& I,
 
 struct HessPlan {
     int nb;        // ceil(C / 256)
-    int tiles;     // nb (nb + 1) / 2
+    int tiles;     // T = nb (nb + 1) / 2
     int kblocks;   // ceil(n / 128): pipeline stages over the calibration rows
-    int split;     // S
+    int split0;    // first tile cut into parts (T when none is)
+    int split;     // parts of the tiles from split0 on (1 when none is cut)
+    int units;     // CTA pairs: (split0 whole tiles) + (T - split0) * split
 };
 
 __host__ __device__ inline HessPlan hess_plan(int64_t n, int64_t C) {
@@ -110,11 +120,31 @@ __host__ __device__ inline HessPlan hess_plan(int64_t n, int64_t C) {
     p.nb = static_cast<int>((C + kPTile - 1) / kPTile);
     p.tiles = p.nb * (p.nb + 1) / 2;
     p.kblocks = static_cast<int>((n + kPBK - 1) / kPBK);
-    int s = kPPairsPerGpu / p.tiles;
-    const int cap = p.kblocks / 16;
+    const int cap = p.kblocks / 16;                       // a part holds at least 16 stages
+    const int r = p.tiles <= kPPairsPerGpu ? p.tiles : p.tiles % kPPairsPerGpu;   // tiles of the last wave
+    int s = r > 0 ? kPPairsPerGpu / r : 1;
     if (s > cap) s = cap;
-    p.split = s < 1 ? 1 : s;
+    if (s < 2 || r == 0) {
+        p.split0 = p.tiles;
+        p.split = 1;
+    } else {
+        p.split0 = p.tiles - r;
+        p.split = s;
+    }
+    p.units = p.split0 + (p.tiles - p.split0) * p.split;
     return p;
+}
+
+// Unit u -> (tile, part); the partial's workspace slot is u - split0 (units with one part have none).
+__host__ __device__ __forceinline__ void hess_unit(const HessPlan& p, int u, int& tile, int& part) {
+    if (u < p.split0) {
+        tile = u;
+        part = 0;
+    } else {
+        const int v = u - p.split0;
+        tile = p.split0 + v / p.split;
+        part = v % p.split;
+    }
 }
 
 struct HessParams {
@@ -146,13 +176,14 @@ hessian_pair_kernel(const __grid_constant__ CUtensorMap tmap, const HessParams p
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
     const int unit = static_cast<int>(blockIdx.x >> 1);
-    const int tile = unit / p.plan.split;
-    const int part = unit % p.plan.split;
+    int tile, part;
+    hess_unit(p.plan, unit, tile, part);
+    const int nparts = tile < p.plan.split0 ? 1 : p.plan.split;
     int I, J;
     hess_tile_coords(tile, p.plan.nb, I, J);
     const bool diag = (I == J);
-    const int kb0 = static_cast<int>(static_cast<int64_t>(part) * p.plan.kblocks / p.plan.split);
-    const int kb1 = static_cast<int>(static_cast<int64_t>(part + 1) * p.plan.kblocks / p.plan.split);
+    const int kb0 = static_cast<int>(static_cast<int64_t>(part) * p.plan.kblocks / nparts);
+    const int kb1 = static_cast<int>(static_cast<int64_t>(part + 1) * p.plan.kblocks / nparts);
     const int nk = kb1 - kb0;
     const int nchunks = (nk + kPChunkKB - 1) / kPChunkKB;
 
@@ -282,9 +313,9 @@ hessian_pair_kernel(const __grid_constant__ CUtensorMap tmap, const HessParams p
                 }
                 // ---- final values of columns gj0 .. gj0+31 of row gi
                 const int gj0 = J * kPTile + blk * 32;
-                if (p.plan.split > 1) {
-                    // partial of this part: workspace [unit][column 256][row 256]
-                    float* dst = ws + static_cast<int64_t>(unit) * kPTile * kPTile +
+                if (nparts > 1) {
+                    // partial of this part: workspace [slot][column 256][row 256]
+                    float* dst = ws + static_cast<int64_t>(unit - p.plan.split0) * kPTile * kPTile +
                                  static_cast<int64_t>(blk * 32) * kPTile + row_in_tile;
 #pragma unroll
                     for (int jj = 0; jj < 32; ++jj) dst[jj * kPTile] = __uint_as_float(a[jj]);
@@ -332,14 +363,16 @@ hessian_pair_kernel(const __grid_constant__ CUtensorMap tmap, const HessParams p
     }
 }
 
-// Adds the S partials of every tile in fixed order, scales by 1/n and stores
-// the tile's upper part and its mirror.  One 32x32 block of a tile per CTA of
-// 32x8 threads; the row-major store goes through a shared transpose so both
-// stores are coalesced.
+// Adds the S partials of every tile cut into parts in fixed order, scales by
+// 1/n and stores the tile's upper part and its mirror.  One 32x32 block of a
+// tile per CTA of 32x8 threads (blockIdx.x counts the cut tiles from split0);
+// the row-major store goes through a shared transpose so both stores are
+// coalesced.
 __global__ void __launch_bounds__(256)
 hessian_reduce_kernel(const float* __restrict__ ws, const HessParams p, float* __restrict__ H) {
     __shared__ float blk[32][33];
-    const int tile = blockIdx.x;
+    const int tile = p.plan.split0 + static_cast<int>(blockIdx.x);
+    const int slot0 = static_cast<int>(blockIdx.x) * p.plan.split;
     const int bi = blockIdx.y >> 3;     // 8 x 8 blocks of 32 in a 256 tile
     const int bj = blockIdx.y & 7;
     int I, J;
@@ -354,7 +387,7 @@ hessian_reduce_kernel(const float* __restrict__ ws, const HessParams p, float* _
         const int i = bi * 32 + tx, j = bj * 32 + jj;
         float s = 0.0f;
         for (int part = 0; part < S; ++part)
-            s = __fadd_rn(s, ws[(static_cast<int64_t>(tile) * S + part) * kPTile * kPTile +
+            s = __fadd_rn(s, ws[static_cast<int64_t>(slot0 + part) * kPTile * kPTile +
                                 static_cast<int64_t>(j) * kPTile + i]);
         s *= p.inv_n;
         blk[tx][jj] = s;

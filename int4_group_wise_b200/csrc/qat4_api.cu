@@ -149,7 +149,7 @@ size_t qat4_hessian_workspace_bytes(int64_t n, int64_t C) {
     if (n < 1 || C < 32 || C % 32 != 0 || C > 65536) return 0;
     const qat4::HessPlan plan = qat4::hess_plan(n, C);
     if (plan.split <= 1) return 0;
-    return static_cast<size_t>(plan.tiles) * plan.split * qat4::kPTile * qat4::kPTile * sizeof(float);
+    return static_cast<size_t>(plan.tiles - plan.split0) * plan.split * qat4::kPTile * qat4::kPTile * sizeof(float);
 }
 
 }  // extern "C"
@@ -199,12 +199,12 @@ qat4_status hessian_run(const uint16_t* X, int64_t n, int64_t C, int64_t n_norm,
     // generous bound: 4 s plus 100 ns per calibration row (a chunk of the
     // mainloop takes ~2 ns per row at full rate)
     p.limit_ns = 4000000000ull + 100ull * static_cast<uint64_t>(n);
-    const unsigned ctas = 2u * static_cast<unsigned>(p.plan.tiles) * static_cast<unsigned>(p.plan.split);
+    const unsigned ctas = 2u * static_cast<unsigned>(p.plan.units);
     qat4::hessian_pair_kernel<<<ctas, qat4::kPThreads, qat4::kPSmemBytes, stream>>>(
         tmap, p, H, static_cast<float*>(workspace));
     if (cudaGetLastError() != cudaSuccess) return QAT4_ERR_CUDA;
-    if (p.plan.split > 1) {
-        const dim3 grid(static_cast<unsigned>(p.plan.tiles), 64);
+    if (p.plan.split > 1) {   // the tiles cut into parts
+        const dim3 grid(static_cast<unsigned>(p.plan.tiles - p.plan.split0), 64);
         qat4::hessian_reduce_kernel<<<grid, 256, 0, stream>>>(static_cast<const float*>(workspace), p, H);
     }
     return launch_status();
@@ -769,8 +769,8 @@ extern "C" qat4_status qat4_selftest_bounded_wait(int64_t limit_ns, cudaStream_t
 // this library holds until the process exits.
 namespace {
 
-// Largest workspace the Hessian planner can ask for: n is split only while
-// tiles * S <= 74, and each (tile, part) unit needs one 256 x 256 fp32 partial.
+// Largest workspace the Hessian planner can ask for: at most 74 parts of cut
+// tiles, each one 256 x 256 fp32 partial.
 constexpr size_t kNoallocScratchBytes =
     static_cast<size_t>(qat4::kPPairsPerGpu) * qat4::kPTile * qat4::kPTile * sizeof(float);  // 18.5 MiB
 
