@@ -97,13 +97,28 @@ __device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t saddr) {
     return d;
 }
 
-// Upper-triangle tile t -> (I, J), I <= J, enumerated row by row.
-__host__ __device__ __forceinline__ void hess_tile_coords(int t, int nb, int& I, int& J) {
-    int i = 0;
-    int rowlen = nb;
-    while (t >= rowlen) { t -= rowlen; ++i; --rowlen; }
-    I = i;
-    J = i + t;
+// Upper-triangle tile t -> (I, J), I <= J.  Tiles are numbered in bands of
+// kPBand tile rows: within a band column by column (J ascending), and within a
+// column down the band's rows (I <= J).  74 consecutive tiles -- one wave of
+// SM pairs, which walk the calibration rows together -- then touch about 18
+// column strips of X instead of all of them, so each wave reads less of X from
+// HBM (C = 14336: 56 strips; row-by-row numbering re-read all of X in every
+// wave, 81 GB per Hessian of 131072 rows).
+constexpr int kPBand = 8;
+__host__ __device__ inline void hess_tile_coords(int t, int nb, int& I, int& J) {
+    for (int i0 = 0; i0 < nb; i0 += kPBand) {
+        const int i1 = i0 + kPBand < nb ? i0 + kPBand : nb;   // band rows [i0, i1)
+        for (int j = i0; j < nb; ++j) {
+            const int cnt = (i1 < j + 1 ? i1 : j + 1) - i0;   // rows i0 .. min(i1, j + 1) - 1
+            if (t < cnt) {
+                I = i0 + t;
+                J = j;
+                return;
+            }
+            t -= cnt;
+        }
+    }
+    I = J = 0;   // not reached for t < nb (nb + 1) / 2
 }
 
 struct HessPlan {
