@@ -589,8 +589,21 @@ qat4_status qat4_w4a16_gemv(const uint16_t* x, int64_t M, const uint8_t* packed,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return QAT4_ERR_CUDA;
     }
-    if (cudaMemsetAsync(y, 0, static_cast<size_t>(M) * static_cast<size_t>(R) * sizeof(float), stream) != cudaSuccess)
-        return QAT4_ERR_CUDA;
+    // both launches may overlap the previous kernel of the stream (programmatic dependent launch);
+    // each waits for it before it reads x or writes y
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    {
+        const int64_t ny = M * R;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>((ny / 4 + 255) / 256 + 1, 4 * info->sms)));
+        cfg.blockDim = dim3(256);
+        cfg.stream = stream;
+        cfg.attrs = pdl;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, qat4::gemv_zero_kernel, y, ny) != cudaSuccess) return QAT4_ERR_CUDA;
+    }
     qat4::GemvParams p;
     p.scales = scales;
     p.R = static_cast<int>(R);
@@ -620,8 +633,14 @@ qat4_status qat4_w4a16_gemv(const uint16_t* x, int64_t M, const uint8_t* packed,
         p.MT = mt;
         p.x = x + m0 * C;
         p.y = y + m0 * R;
-        qat4::w4a16_gemv_kernel<<<grid, qat4::kGmThreads, qat4::gemv_smem_bytes(mt, c, stages), stream>>>(tmap, p);
-        if (cudaGetLastError() != cudaSuccess) return QAT4_ERR_CUDA;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(grid));
+        cfg.blockDim = dim3(qat4::kGmThreads);
+        cfg.dynamicSmemBytes = qat4::gemv_smem_bytes(mt, c, stages);
+        cfg.stream = stream;
+        cfg.attrs = pdl;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, qat4::w4a16_gemv_kernel, tmap, p) != cudaSuccess) return QAT4_ERR_CUDA;
     }
     return QAT4_OK;
 }

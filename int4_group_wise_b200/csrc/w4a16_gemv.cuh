@@ -163,8 +163,41 @@ __device__ __forceinline__ void gm_scales(const GmScaleCtx& x, int b, int ch, fl
     }
 }
 
+// Programmatic dependent launch.  Calls of the product on one stream are
+// launched so that the next kernel may start while this one finishes: the
+// next call's CTAs become resident as this one's retire and start streaming
+// their (constant) codes, and wait for this kernel's completion only before
+// they read x or touch y.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Returns when the kernel this one depends on (the previous one in the stream)
+// has completed and its writes are visible; at once if there is none.
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Zeroes y (the row blocks cut between two CTAs get two atomic partials), in
+// order: it may start early, but writes y only after the previous kernel of
+// the stream -- which may still be reading or adding into the same buffer --
+// has completed.
+__global__ void __launch_bounds__(256)
+gemv_zero_kernel(float* __restrict__ y, int64_t n) {
+    pdl_launch_dependents();
+    pdl_wait();
+    const int64_t n4 = n >> 2;
+    float4* y4 = reinterpret_cast<float4*>(y);
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        y4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int64_t i = (n4 << 2) + static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        y[i] = 0.0f;
+}
+
 __global__ void __launch_bounds__(kGmThreads)
 w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tmap, const GemvParams p) {
+    pdl_launch_dependents();
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;          // the swizzle needs 1 KB alignment
@@ -232,6 +265,8 @@ w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tmap, const GemvParams p) 
     }
 
     // -------------------------------------------------------------- consumers
+    // x (and y) belong to the stream's order: wait for the kernel before this one
+    pdl_wait();
     // stage x once: token m's word w (columns 8w..8w+7) in the order 0,4,1,5,2,6,3,7; columns
     // past C are zero
     {
