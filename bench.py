@@ -953,19 +953,27 @@ def run_fq_gemm(args):
         torch.cuda.synchronize()
         return sorted(a.elapsed_time(b) for a, b in ts)
 
-    fused = lambda: q4.fq_gemm(X, W, D, Y)
+    ws = torch.empty(q4.lib().qat4_fq_gemm_staged_workspace_bytes(R, C), dtype=torch.uint8, device=dev)
+    staged = lambda: q4.fq_gemm(X, W, D, Y, workspace=ws)
+    fused = lambda: q4.fq_gemm(X, W, D, Y, fused=True)
 
     def unfused():
         q4.lsq_fwd(W, D, Q)
         torch.matmul(X, Q.to(torch.bfloat16).t())
 
     for _ in range(args.warmup):
+        staged()
         fused()
         unfused()
     q4.sync_check()
+    # interleaved rounds so that the three paths see the same power state
+    t_f, t_1, t_u = [], [], []
     with ClockSampler(0) as clk:
-        t_f = timed(fused, args.steps)
-    t_u = timed(unfused, max(3, args.steps // 2))
+        for _ in range(3):
+            t_f += timed(staged, max(1, args.steps // 3))
+            t_1 += timed(fused, max(1, args.steps // 3))
+            t_u += timed(unfused, max(1, args.steps // 3))
+    t_f.sort()
     q4.sync_check()
     flop = 2.0 * T * R * C
     ms = statistics.median(t_f)
@@ -980,9 +988,11 @@ def run_fq_gemm(args):
         "roofline": {"bound": "tensor", "achieved": tf, "peak": peak, "unit": "TFLOP/s", "frac": tf / peak,
                      "flop_per_launch": flop, "peak_kind": f"{peak_kind} bf16 burst"},
         "ms_min_median_max": [t_f[0], ms, t_f[-1]],
+        "what": "qat4_fq_gemm_staged: quantizer into a bf16 workspace, then a persistent tcgen05 GEMM",
+        "fused_single_kernel_ms": statistics.median(t_1),
         "unfused_library_ms": statistics.median(t_u),
         "unfused_library": "qat4_lsq_fwd + cast to bf16 + torch.matmul (cuBLAS bf16), same product",
-        "gpu_launches": args.steps, "clocks": clk.summary()}), flush=True)
+        "gpu_launches": 2 * len(t_f), "clocks": clk.summary()}), flush=True)
 
 
 def run_hessian_split(args):

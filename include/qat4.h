@@ -339,6 +339,21 @@ qat4_status qat4_w4a16_gemv(const uint16_t *x, int64_t M, const uint8_t *packed,
 qat4_status qat4_fq_gemm(const uint16_t *X, int64_t T, const float *W, const float *delta, int64_t R, int64_t C,
                          float *Y, cudaStream_t stream);
 
+/* The same product in two kernels: the quantizer writes bf16(Q_Delta(W))
+ * (the same values the fused call forms in shared memory) into `workspace`,
+ * then a persistent tcgen05 GEMM computes Y = X * Qb^T.  Arguments as for
+ * qat4_fq_gemm, plus
+ *  workspace  device scratch of at least
+ *             qat4_fq_gemm_staged_workspace_bytes(R, C) bytes (R * C bf16,
+ *             rounded up to 256), 256-byte aligned; contents on entry are
+ *             ignored, on return it holds bf16(Q_Delta(W)) [R, C].
+ *  Same result as qat4_fq_gemm up to the order of the float32 sums.
+ *  Errors: QAT4_ERR_NULL, _SHAPE, _ALIGN, _WORKSPACE, _CUDA; a bounded wait
+ *  that gives up leaves QAT4_ERR_TIMEOUT for qat4_sync_check. */
+size_t qat4_fq_gemm_staged_workspace_bytes(int64_t R, int64_t C);
+qat4_status qat4_fq_gemm_staged(const uint16_t *X, int64_t T, const float *W, const float *delta, int64_t R,
+                                int64_t C, float *Y, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the library's device error
  * word for the current device.  Returns QAT4_ERR_TIMEOUT if a kernel gave up
  * a bounded wait since the last check, QAT4_ERR_CUDA if synchronisation

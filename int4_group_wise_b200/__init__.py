@@ -51,6 +51,8 @@ EXPORTS = {
     "qat4_scale_search_rowwise": (ct.c_int, [_P, _I64, _I64, _P, _I64, _P, _I32, _P, _P, _P, _P, _Z, _P]),
     "qat4_w4a16_gemv": (ct.c_int, [_P, _I64, _P, _P, _I64, _I64, _I64, _P, _P]),
     "qat4_fq_gemm": (ct.c_int, [_P, _I64, _P, _P, _I64, _I64, _P, _P]),
+    "qat4_fq_gemm_staged_workspace_bytes": (ct.c_size_t, [_I64, _I64]),
+    "qat4_fq_gemm_staged": (ct.c_int, [_P, _I64, _P, _P, _I64, _I64, _P, _P, ct.c_size_t, _P]),
     "qat4_refine_workspace_bytes": (ct.c_size_t, [_I64, _I64]),
     "qat4_refine": (ct.c_int, [_P, _I64, _I64, _P, _I64, _P, ct.c_int32, ct.c_int32, _P, _P, _P, _P, _Z, _P]),
     "qat4_sync_check": (ct.c_int, [_P]),
@@ -430,9 +432,11 @@ def w4a16_gemv(x, packed, scales, y=None, stream=None):
     return y
 
 
-def fq_gemm(X, W, delta, Y=None, stream=None):
+def fq_gemm(X, W, delta, Y=None, stream=None, fused=False, workspace=None):
     """Y [T, R] float32 = X @ bf16(Q_delta(W))^T; X bf16 [T, C], W float32 [R, C], delta float32
-    [R, C/32]."""
+    [R, C/32].  By default the staged call (the quantizer writes bf16 Q into `workspace`, allocated
+    here when None, then a tcgen05 GEMM); fused=True runs the single kernel with the quantizer in
+    the GEMM's producer (no workspace)."""
     import torch
     L = lib()
     _dev(X, "X", torch.bfloat16)
@@ -443,8 +447,16 @@ def fq_gemm(X, W, delta, Y=None, stream=None):
         raise ValueError("W must be [R, C] with the C of X")
     _dev(delta, "delta", torch.float32, (R, C // 32))
     Y = _out(Y, "Y", (T, R), torch.float32, X)
-    _check(L.qat4_fq_gemm(_dev(X, "X"), T, _dev(W, "W"), _dev(delta, "delta"), R, C, _dev(Y, "Y"),
-                          _stream(stream)), "qat4_fq_gemm")
+    if fused:
+        _check(L.qat4_fq_gemm(_dev(X, "X"), T, _dev(W, "W"), _dev(delta, "delta"), R, C, _dev(Y, "Y"),
+                              _stream(stream)), "qat4_fq_gemm")
+        return Y
+    need = int(L.qat4_fq_gemm_staged_workspace_bytes(R, C))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    _check(L.qat4_fq_gemm_staged(_dev(X, "X"), T, _dev(W, "W"), _dev(delta, "delta"), R, C, _dev(Y, "Y"),
+                                 _dev(workspace, "workspace"), workspace.numel(), _stream(stream)),
+           "qat4_fq_gemm_staged")
     return Y
 
 

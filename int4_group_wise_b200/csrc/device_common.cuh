@@ -23,6 +23,9 @@ constexpr float kQmax = 7.0f;
 
 enum : int { QAT4_DEV_ERR_TIMEOUT = 1 };
 
+// Bound of the waits that drain a CTA's copies and MMAs in flight before it exits.
+constexpr uint64_t kDrainLimitNs = 1000000000ull;
+
 // Device error word (one per device, per loaded copy of the library).
 __device__ int g_dev_error;
 
@@ -348,6 +351,18 @@ __device__ __forceinline__ uint32_t tmem_ld_32x32b_x1(uint32_t taddr) {
 }
 __device__ __forceinline__ void tmem_ld_wait() {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ------------------------------------------------ programmatic dependent launch
+// Lets the next kernel of the stream (launched with programmatic stream
+// serialization) start before this one completes.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Returns when the kernel this one depends on (the previous one in the stream)
+// has completed and its writes are visible; at once if there is none.
+__device__ __forceinline__ void pdl_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ------------------------------------------------------- quantizer primitive

@@ -170,7 +170,6 @@ struct HessParams {
     uint64_t limit_ns;   // bounded-wait limit
 };
 
-constexpr uint64_t kDrainLimitNs = 1000000000ull;   // bounded drain on the error path
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPThreads, 1)
 hessian_pair_kernel(const __grid_constant__ CUtensorMap tmap, const HessParams p,

@@ -21,6 +21,7 @@
 #include "rowwise_search.cuh"
 #include "w4a16_gemv.cuh"
 #include "fq_gemm.cuh"
+#include "fq_staged.cuh"
 #include "refine.cuh"
 
 namespace {
@@ -42,6 +43,7 @@ struct DeviceInfo {
     bool rowsearch_attr = false;
     int smem_optin = 0;       // opt-in shared memory per block; gemv attributes set when > 0
     bool fq_attr = false;
+    bool gemm_attr = false;
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_mutex;
@@ -702,6 +704,101 @@ qat4_status qat4_fq_gemm(const uint16_t* X, int64_t T, const float* W, const flo
     p.limit_ns = 4000000000ull + 10000ull * static_cast<uint64_t>(p.ksteps);
     const unsigned grid = static_cast<unsigned>(2 * tiles_m * tiles_r);
     qat4::fq_gemm_kernel<<<grid, qat4::kFqThreads, qat4::kFqSmemBytes, stream>>>(tx, tw, p);
+    return launch_status();
+}
+
+size_t qat4_fq_gemm_staged_workspace_bytes(int64_t R, int64_t C) {
+    if (!valid_rc(R, C)) return 0;
+    return (static_cast<size_t>(R) * static_cast<size_t>(C) * 2 + 255) & ~size_t(255);
+}
+
+qat4_status qat4_fq_gemm_staged(const uint16_t* X, int64_t T, const float* W, const float* delta, int64_t R,
+                                int64_t C, float* Y, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (!X || !W || !delta || !Y || !workspace) return QAT4_ERR_NULL;
+    if (T < 1 || T > (int64_t(1) << 31) - 1 || !valid_rc(R, C) || T * R > (int64_t(1) << 40)) return QAT4_ERR_SHAPE;
+    if (!aligned16(X) || !aligned16(W) || !aligned16(delta) || !aligned16(Y) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return QAT4_ERR_ALIGN;
+    if (workspace_bytes < qat4_fq_gemm_staged_workspace_bytes(R, C)) return QAT4_ERR_WORKSPACE;
+    const int64_t tiles_m = (T + qat4::kGTile - 1) / qat4::kGTile;
+    const int64_t tiles_n = (R + qat4::kGTile - 1) / qat4::kGTile;
+    if (tiles_m * tiles_n > (int64_t(1) << 31) - 1) return QAT4_ERR_SHAPE;
+    int dev = 0;
+    DeviceInfo* info = nullptr;
+    if (!device_info(&dev, &info)) return QAT4_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lock(g_mutex);
+        if (!info->gemm_attr) {
+            if (cudaFuncSetAttribute(qat4::gemm_bf16_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(qat4::kGSmemBytes)) != cudaSuccess)
+                return QAT4_ERR_CUDA;
+            info->gemm_attr = true;
+        }
+    }
+    EncodeTiledFn encode = encode_tiled();
+    if (!encode) return QAT4_ERR_CUDA;
+    uint16_t* Qb = static_cast<uint16_t*>(workspace);
+    // both operands bf16 K-major [rows, C]: one box = 128 rows x 64 columns (128 bytes), 128-byte swizzle
+    CUtensorMap ta, tb;
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(qat4::kGHalf)};
+    const cuuint32_t estr[2] = {1, 1};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(C) * 2};
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(T)};
+        if (encode(&ta, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(X), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return QAT4_ERR_CUDA;
+    }
+    {
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(C), static_cast<cuuint64_t>(R)};
+        if (encode(&tb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, Qb, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return QAT4_ERR_CUDA;
+    }
+    CUtensorMap ty = {};
+    const bool tma_store = (R % 4) == 0;     // rows of Y 16-byte aligned
+    if (tma_store) {   // Y float32 [T, R]: one box = 32 rows x 32 columns (128 bytes), 128-byte swizzle
+        const cuuint64_t dims[2] = {static_cast<cuuint64_t>(R), static_cast<cuuint64_t>(T)};
+        const cuuint64_t ystr[1] = {static_cast<cuuint64_t>(R) * 4};
+        const cuuint32_t ybox[2] = {32, 32};
+        if (encode(&ty, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, Y, dims, ystr, ybox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return QAT4_ERR_CUDA;
+    }
+    // 1. Qb = bf16(Q_Delta(W)), 16 weights per thread
+    const int64_t nhalf = R * C / 16;
+    qat4::fq_quantize_kernel<<<static_cast<unsigned>((nhalf + qat4::kFqQuantBlock - 1) / qat4::kFqQuantBlock),
+                               qat4::kFqQuantBlock, 0, stream>>>(W, delta, nhalf, Qb);
+    if (cudaGetLastError() != cudaSuccess) return QAT4_ERR_CUDA;
+    // 2. Y = X Qb^T on the tensor cores, one persistent pair per SM pair
+    qat4::GemmParams p;
+    p.Y = Y;
+    p.T = static_cast<int>(T);
+    p.R = static_cast<int>(R);
+    p.C = static_cast<int>(C);
+    p.tiles_m = static_cast<int>(tiles_m);
+    p.tiles = static_cast<int>(tiles_m * tiles_n);
+    p.ksteps = static_cast<int>((C + qat4::kGBK - 1) / qat4::kGBK);
+    p.tma_store = tma_store ? 1 : 0;
+    const int pairs = static_cast<int>(std::min<int64_t>(qat4::kGPairsPerGpu, tiles_m * tiles_n));
+    const int64_t per_pair = (tiles_m * tiles_n + pairs - 1) / pairs;
+    // generous bound: 4 s plus 10 us per 128-column step of a pair's tiles (a step takes well under 1 us)
+    p.limit_ns = 4000000000ull + 10000ull * static_cast<uint64_t>(per_pair * p.ksteps);
+    // launched early (programmatic dependent launch): its producer waits for the quantizer
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    cfg.blockDim = dim3(qat4::kGThreads);
+    cfg.dynamicSmemBytes = qat4::kGSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, qat4::gemm_bf16_pair_kernel, ta, tb, ty, p) != cudaSuccess) return QAT4_ERR_CUDA;
     return launch_status();
 }
 

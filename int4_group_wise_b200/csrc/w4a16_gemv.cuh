@@ -163,19 +163,12 @@ __device__ __forceinline__ void gm_scales(const GmScaleCtx& x, int b, int ch, fl
     }
 }
 
-// Programmatic dependent launch.  Calls of the product on one stream are
-// launched so that the next kernel may start while this one finishes: the
-// next call's CTAs become resident as this one's retire and start streaming
-// their (constant) codes, and wait for this kernel's completion only before
-// they read x or touch y.
-__device__ __forceinline__ void pdl_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-// Returns when the kernel this one depends on (the previous one in the stream)
-// has completed and its writes are visible; at once if there is none.
-__device__ __forceinline__ void pdl_wait() {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-}
+// Programmatic dependent launch (pdl_launch_dependents / pdl_wait in
+// device_common.cuh).  Calls of the product on one stream are launched so that
+// the next kernel may start while this one finishes: the next call's CTAs
+// become resident as this one's retire and start streaming their (constant)
+// codes, and wait for this kernel's completion only before they read x or
+// touch y.
 
 // Zeroes y (the row blocks cut between two CTAs get two atomic partials), in
 // order: it may start early, but writes y only after the previous kernel of

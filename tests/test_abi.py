@@ -109,6 +109,12 @@ def test_fq_gemm_validation():
     assert L.qat4_fq_gemm(A, 8, A, A, 0, 64, A, None) == 2
     assert L.qat4_fq_gemm(A, 8, MIS, A, 8, 64, A, None) == 3
     assert L.qat4_fq_gemm(A, 8, A, A, 8, 64, MIS, None) == 3
+    need = L.qat4_fq_gemm_staged_workspace_bytes(8, 64)
+    assert need == 1024
+    assert L.qat4_fq_gemm_staged(A, 8, A, A, 8, 64, A, None, need, None) == 1
+    assert L.qat4_fq_gemm_staged(A, 8, A, A, 8, 48, A, A, need, None) == 2
+    assert L.qat4_fq_gemm_staged(A, 8, A, A, 8, 64, A, MIS, need, None) == 3
+    assert L.qat4_fq_gemm_staged(A, 8, A, A, 8, 64, A, A, need - 256, None) == 5
 
 
 def test_hessian_partial_validation():

@@ -1,5 +1,6 @@
-"""GPU parity of the fused fake-quant forward GEMM Y = X bf16(Q_Delta(W))^T against the binary64
-oracle.  The operand bf16(Q) is formed on the GPU from the same code decision as the oracle;
+"""GPU parity of the fake-quant forward GEMM Y = X bf16(Q_Delta(W))^T against the binary64
+oracle, for both calls: the staged one (quantizer, then a persistent tcgen05 GEMM) and the fused
+one (the quantizer in the GEMM's producer).  The operand bf16(Q) is formed on the GPU from the same code decision as the oracle;
 products of bf16 values are exact in float32, so the only difference is the float32 summation
 of C products: |Y - Y_ref| <= C * 2^-23 * sum_c |x_c| |b_c| (the classical bound for a
 recursively summed dot product, doubled to cover a truncating accumulator)."""
@@ -24,9 +25,9 @@ def _problem(T, R, C, seed):
     return Xb, W, D
 
 
-def _run(Xb, W, D):
+def _run(Xb, W, D, fused=False):
     tX = torch.from_numpy(Xb.view(np.int16)).cuda().view(torch.bfloat16)
-    Y = q4.fq_gemm(tX, torch.from_numpy(W).cuda(), torch.from_numpy(D).cuda())
+    Y = q4.fq_gemm(tX, torch.from_numpy(W).cuda(), torch.from_numpy(D).cuda(), fused=fused)
     q4.sync_check()
     return Y.cpu().numpy().astype(np.float64)
 
@@ -39,33 +40,38 @@ def _abs_bound(Xb, W, D, tt=None, rr=None):
     return np.einsum("mc,mc->m", ax[tt], np.abs(Qb[rr]))
 
 
+@pytest.mark.parametrize("fused", [False, True])
 @pytest.mark.parametrize("T,R,C", [(256, 256, 64), (1, 33, 32), (300, 300, 96), (513, 257, 2080),
-                                   (128, 512, 4096), (260, 1000, 512)])
-def test_fq_gemm_matches_oracle(T, R, C, oracle_mod):
-    """Single and multiple 256x256 tiles, ragged tokens, rows and columns (C % 64 == 32)."""
+                                   (128, 512, 4096), (260, 1000, 512), (2048, 2560, 384), (600, 19030, 160)])
+def test_fq_gemm_matches_oracle(T, R, C, fused, oracle_mod):
+    """Single and multiple 256x256 tiles (more tiles than SM pairs in the last two, so the staged
+    GEMM's pairs take several tiles and alternate accumulators), ragged tokens, rows (R % 4 != 0)
+    and columns (C % 128 == 32 or 96)."""
     Xb, W, D = _problem(T, R, C, seed=T + R + C)
-    Y = _run(Xb, W, D)
+    Y = _run(Xb, W, D, fused)
     Yr = oracle_mod.fq_gemm(Xb, W, D)
     bound = C * 2.0 ** -23 * _abs_bound(Xb, W, D) + 1e-30
     err = np.abs(Y - Yr)
     assert np.all(err <= bound), float(np.max(err / bound))
 
 
-def test_fq_gemm_zero_groups_and_clamps(oracle_mod):
+@pytest.mark.parametrize("fused", [False, True])
+def test_fq_gemm_zero_groups_and_clamps(fused, oracle_mod):
     """All-zero groups (Delta = 0) give Q = 0; scales far below max|w|/7 clamp most codes."""
     T, R, C = 256, 256, 128
     Xb, W, D = _problem(T, R, C, seed=5)
     W[:, 32:64] = 0.0
     D[:, 1] = 0.0
     D[:, 2] *= f32(0.1)
-    Y = _run(Xb, W, D)
+    Y = _run(Xb, W, D, fused)
     Yr = oracle_mod.fq_gemm(Xb, W, D)
     bound = C * 2.0 ** -23 * _abs_bound(Xb, W, D) + 1e-30
     assert np.all(np.abs(Y - Yr) <= bound)
 
 
 @pytest.mark.slow
-def test_fq_gemm_up_projection_full_size(oracle_mod):
+@pytest.mark.parametrize("fused", [False, True])
+def test_fq_gemm_up_projection_full_size(fused, oracle_mod):
     """The 1B-class up-projection (W 8192x2048) on a micro-batch of 8192 tokens, the size the
     benchmark times; 4096 sampled outputs against the oracle."""
     wl = inputs.workload(1)
@@ -75,7 +81,7 @@ def test_fq_gemm_up_projection_full_size(oracle_mod):
     D = (np.abs(W).reshape(W.shape[0], -1, 32).max(axis=2) / f32(7) *
          rng.uniform(0.5, 1.0, (W.shape[0], W.shape[1] // 32))).astype(f32)
     Xb = wl.activations(m.x_name, n=8192)
-    Y = _run(Xb, W, D)
+    Y = _run(Xb, W, D, fused)
     tt = rng.integers(0, Xb.shape[0], 4096)
     rr = rng.integers(0, W.shape[0], 4096)
     ref = oracle_mod.fq_gemm_entries(Xb, W, D, tt, rr)
@@ -83,13 +89,18 @@ def test_fq_gemm_up_projection_full_size(oracle_mod):
     assert np.all(np.abs(Y[tt, rr] - ref) <= bound)
 
 
-def test_fq_gemm_deterministic():
+@pytest.mark.parametrize("fused", [False, True])
+def test_fq_gemm_deterministic(fused):
     """Repeated launches give bitwise identical Y (the ring slots are reused only after their
-    contents are consumed; a race there shows up as whole W rows differing)."""
+    contents are consumed; a race there shows up as whole W rows differing), and both calls give
+    the same products up to the float32 summation order."""
     Xb, W, D = _problem(1024, 2048, 2048, seed=9)
     tX = torch.from_numpy(Xb.view(np.int16)).cuda().view(torch.bfloat16)
     tW, tD = torch.from_numpy(W).cuda(), torch.from_numpy(D).cuda()
-    Y0 = q4.fq_gemm(tX, tW, tD).clone()
+    Y0 = q4.fq_gemm(tX, tW, tD, fused=fused).clone()
     for _ in range(30):
-        assert torch.equal(q4.fq_gemm(tX, tW, tD), Y0)
+        assert torch.equal(q4.fq_gemm(tX, tW, tD, fused=fused), Y0)
+    Y1 = q4.fq_gemm(tX, tW, tD, fused=not fused)
     q4.sync_check()
+    bound = 2048 * 2.0 ** -22 * torch.from_numpy(_abs_bound(Xb, W, D)).cuda()
+    assert torch.all((Y1.double() - Y0.double()).abs() <= bound)
