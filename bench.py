@@ -356,8 +356,38 @@ def time_problem(p: DeviceProblem, q4, steps: int, warmup: int, flush: bool, wor
     q4.sync_check()
     mean = {s: sum(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(steps)) / steps
             for i, s in enumerate(STAGES)}
+    floor = copy_floor(p, stage_fn, stream, flush_buf, sink, steps) if flush else None
     del flush_buf
-    return {"total_ms": start.elapsed_time(stop), "stage_ms": mean, "clocks": clk.summary()}
+    return {"total_ms": start.elapsed_time(stop), "stage_ms": mean, "clocks": clk.summary(), "copy_floor": floor}
+
+
+def copy_floor(p: DeviceProblem, stage_fn, stream, flush_buf, sink, steps: int):
+    """Reference for the single-launch streaming stages of a single-layer step: the same steps
+    again, with the LSQ and export launches replaced by a device copy (torch's copy kernel, src ->
+    dst) that moves the stage's algorithmic bytes (half read, half written), after the same L2
+    flush and after the same Hessian and search launches, so that it runs in the same power
+    state.  Returns the mean CUDA-event time of each copy in ms."""
+    import torch
+    units = p.units()
+    bufs = {}
+    for s in ("lsq_fwd_bwd", "pack_w4a16"):
+        half = int(units[s] // 2) // 16 * 16
+        bufs[s] = (torch.ones(half, dtype=torch.uint8, device=p.dev), torch.empty(half, dtype=torch.uint8, device=p.dev))
+    tot = {s: 0.0 for s in bufs}
+    for k in range(steps + 1):                    # the first pass is a warm-up
+        for name in ("hessian", "scale_search"):
+            torch.sum(flush_buf, dim=0, out=sink)
+            stage_fn[name]()
+        for s, (src, dst) in bufs.items():
+            torch.sum(flush_buf, dim=0, out=sink)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            dst.copy_(src)
+            b.record(stream)
+            b.synchronize()
+            if k > 0:
+                tot[s] += a.elapsed_time(b)
+    return {s: tot[s] / steps for s in bufs}
 
 
 def stage_lines(p: DeviceProblem, res, world: int, peaks, peak_kind: str, long_step: bool, traffic: dict):
@@ -388,12 +418,20 @@ def stage_lines(p: DeviceProblem, res, world: int, peaks, peak_kind: str, long_s
                                         "peak": alu_peak / 1e12, "unit": "Top/s", "frac": v / world / search_roof,
                                         "ops_per_group": SEARCH_OPS_PER_CAND * p.K, "groups_per_step": units["scale_search"],
                                         "peak_kind": f"148 SM x 128 FP32 lanes x {sm_max:.0f} MHz"}}
+    floor = res.get("copy_floor")
     for s in ("lsq_fwd_bwd", "pack_w4a16"):
         u, ms = job[s]
         v = u / ms / 1e6
         out[s] = {"value": v, "unit": "GB/s", "ms": ms, "launches": len(p.mats),
                   "roofline": {"bound": "hbm", "achieved": v / world, "peak": hbm, "unit": "GB/s",
                                "frac": v / world / hbm, "bytes_per_step": units[s], "peak_kind": f"{peak_kind} copy"}}
+        if floor is not None:
+            fu, fms = aggregate_over_ranks(units[s], floor[s])
+            fv = fu / fms / 1e6
+            out[s]["copy_floor"] = {
+                "what": "device copy of the same bytes (half read, half written) at the same point of the "
+                        "step (after the flush, the Hessian and the search), CUDA-event timed",
+                "ms": fms, "gbs": fv / world, "frac_of_peak": fv / world / hbm, "stage_over_copy": v / fv}
     for s in STAGES:
         t = traffic.get(s)
         out[s]["roofline"]["traffic"] = t["bytes"] if t else None
