@@ -357,8 +357,35 @@ def time_problem(p: DeviceProblem, q4, steps: int, warmup: int, flush: bool, wor
     mean = {s: sum(evs[k][i][0].elapsed_time(evs[k][i][1]) for k in range(steps)) / steps
             for i, s in enumerate(STAGES)}
     floor = copy_floor(p, stage_fn, stream, flush_buf, sink, steps) if flush else None
+    alone = stages_alone(stage_fn, stream, flush_buf, sink, steps) if flush else None
     del flush_buf
-    return {"total_ms": start.elapsed_time(stop), "stage_ms": mean, "clocks": clk.summary(), "copy_floor": floor}
+    return {"total_ms": start.elapsed_time(stop), "stage_ms": mean, "clocks": clk.summary(), "copy_floor": floor,
+            "alone_ms": alone}
+
+
+def stages_alone(stage_fn, stream, flush_buf, sink, steps: int):
+    """Each stage of a single-layer step on its own: after a 0.2 s pause (the GPU leaves the
+    power state that the previous stage's work put it in), two untimed launches, then `steps`
+    launches, each after the L2 flush and bracketed by CUDA events.  Lightest stage first.
+    Returns {stage: mean ms}."""
+    import torch
+    out = {}
+    for name in ("pack_w4a16", "lsq_fwd_bwd", "scale_search", "hessian"):
+        torch.cuda.synchronize()
+        time.sleep(0.2)
+        for _ in range(2):
+            stage_fn[name]()
+        tot = 0.0
+        for _ in range(steps):
+            torch.sum(flush_buf, dim=0, out=sink)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            stage_fn[name]()
+            b.record(stream)
+            b.synchronize()
+            tot += a.elapsed_time(b)
+        out[name] = tot / steps
+    return out
 
 
 def copy_floor(p: DeviceProblem, stage_fn, stream, flush_buf, sink, steps: int):
@@ -432,6 +459,14 @@ def stage_lines(p: DeviceProblem, res, world: int, peaks, peak_kind: str, long_s
                 "what": "device copy of the same bytes (half read, half written) at the same point of the "
                         "step (after the flush, the Hessian and the search), CUDA-event timed",
                 "ms": fms, "gbs": fv / world, "frac_of_peak": fv / world / hbm, "stage_over_copy": v / fv}
+    alone = res.get("alone_ms")
+    if alone is not None:
+        for s in STAGES:
+            au, ams = aggregate_over_ranks(units[s], alone[s])
+            frac = out[s]["roofline"]["frac"] * out[s]["ms"] / ams     # same work, same peak
+            out[s]["alone"] = {"what": "the stage's launch on its own (after a 0.2 s pause, L2 flushed before "
+                                       "each launch, no other stage in between), CUDA-event timed",
+                               "ms": ams, "frac": frac}
     for s in STAGES:
         t = traffic.get(s)
         out[s]["roofline"]["traffic"] = t["bytes"] if t else None
