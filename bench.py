@@ -984,11 +984,12 @@ def run_w4a16_decode(args):
 
 
 def run_fq_gemm(args):
-    """The fused fake-quant forward GEMM of a QAT step on the 1B-class up-projection (W fp32
-    8192x2048, searched-range scales) for a micro-batch of --tokens tokens: TFLOP/s against the
-    bf16 tensor peak, each launch timed with CUDA events after an L2 flush.  For context the
-    same product is also timed unfused through libraries: the LSQ forward, a cast to bf16 and a
-    cuBLAS bf16 GEMM."""
+    """The fake-quant forward GEMM of a QAT step on the 1B-class up-projection (W fp32 8192x2048,
+    searched-range scales) for a micro-batch of --tokens tokens: TFLOP/s of the staged call
+    (quantizer into a bf16 workspace, then the persistent tcgen05 GEMM) against the bf16 tensor
+    peak, each launch timed with CUDA events after an L2 flush.  Timed beside it, interleaved:
+    the single fused kernel, and the same product unfused through libraries (the LSQ forward, a
+    cast to bf16 and a cuBLAS bf16 GEMM)."""
     import torch
 
     import int4_group_wise_b200 as q4
@@ -1053,7 +1054,7 @@ def run_fq_gemm(args):
     tf = flop / ms / 1e9
     peak = float(peaks["bf16_tflops"])
     print(json.dumps({
-        "metric": "fused fake-quant GEMM TFLOP/s (Y = X bf16(Q_Delta(W))^T)", "value": tf, "unit": "TFLOP/s",
+        "metric": "fake-quant GEMM TFLOP/s (Y = X bf16(Q_Delta(W))^T)", "value": tf, "unit": "TFLOP/s",
         "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "variant": "fq-gemm", "data": "synthetic", "dtype": "bf16 x bf16 -> f32 (quantizer f32)",
         "config": {"workload": f"1B-class up-projection W fp32 {R}x{C}, X bf16 {T}x{C} (micro-batch of {T} tokens)",
@@ -1231,7 +1232,7 @@ def main():
                     default="path",
                     help="per-channel: time the one-scale-per-row LSQ step and export instead; "
                          "w4a16-decode: time the inference GEMV on the packed 8B-class stack; "
-                         "fq-gemm: time the fused fake-quant forward GEMM; "
+                         "fq-gemm: time the fake-quant forward GEMM (staged, fused and unfused); "
                          "hessian-split: the calibration Hessian with its rows split over the ranks; "
                          "refine: one sweep of the full-objective refinement")
     ap.add_argument("--tokens", type=int, default=8192, help="fq-gemm: tokens of the micro-batch")
