@@ -812,7 +812,7 @@ qat4_status qat4_refine(const float* W, int64_t R, int64_t C, const float* H, in
                         int32_t K, int32_t sweeps, int32_t* idx, float* delta, double* obj, void* workspace,
                         size_t workspace_bytes, cudaStream_t stream) {
     if (!W || !H || !alpha || !idx || !delta) return QAT4_ERR_NULL;
-    if (!valid_rc(R, C) || K < 1 || sweeps < 0 || ldh < C || R > 65535 * int64_t(qat4::kRfTile))
+    if (!valid_rc(R, C) || K < 1 || sweeps < 0 || ldh < C || R > 65535 * int64_t(qat4::kRfTileR))
         return QAT4_ERR_SHAPE;
     if (!aligned16(W) || !aligned16(H) || !aligned16(alpha) || !aligned16(idx) || !aligned16(delta) ||
         (obj && !aligned16(obj)) || (ldh % 4) != 0 || (workspace && !aligned16(workspace)))
@@ -829,8 +829,8 @@ qat4_status qat4_refine(const float* W, int64_t R, int64_t C, const float* H, in
     const unsigned eb = static_cast<unsigned>(err_blocks < int64_t(info->sms) * 16 ? err_blocks : int64_t(info->sms) * 16);
     qat4::refine_err_kernel<<<eb, 256, 0, stream>>>(W, ngroups, alpha, K, idx, E);
     if (cudaGetLastError() != cudaSuccess) return QAT4_ERR_CUDA;
-    const dim3 vgrid(static_cast<unsigned>((C + qat4::kRfTile - 1) / qat4::kRfTile),
-                     static_cast<unsigned>((R + qat4::kRfTile - 1) / qat4::kRfTile));
+    const dim3 vgrid(static_cast<unsigned>((C + qat4::kRfTileC - 1) / qat4::kRfTileC),
+                     static_cast<unsigned>((R + qat4::kRfTileR - 1) / qat4::kRfTileR));
     qat4::refine_v_kernel<<<vgrid, 256, 0, stream>>>(E, static_cast<int>(R), static_cast<int>(C), H, ldh, V);
     if (cudaGetLastError() != cudaSuccess) return QAT4_ERR_CUDA;
     const unsigned sgrid = static_cast<unsigned>((R + qat4::kRfWarps - 1) / qat4::kRfWarps);

@@ -16,12 +16,15 @@
 //                       (exact: difference of two binary32 values);
 //   refine_v_kernel     V = E H, a tiled binary64 product (H read once per
 //                       64-row tile), into the caller's workspace;
-//   refine_sweep_kernel one warp per row walks the groups: u_g from v and the
-//                       group's block of H; every candidate's
+//   refine_sweep_kernel one warp per row, the CTA's rows walking the groups in
+//                       lockstep: u_g from v and the group's block of H (staged
+//                       once per CTA); every candidate's
 //                       e' H_gg e'^T + 2 e'.u_g in binary64 (lanes take
 //                       candidates k = lane, lane + 32, ...; H_gg folded into
 //                       its upper triangle in shared memory); the warp's
-//                       argmin; when the group moves, v += H[:, g] (e'_g - e_g).
+//                       argmin; for the rows whose group moved,
+//                       v += H[:, g] (e'_g - e_g), with each of the group's 32
+//                       rows of H read once for the whole CTA.
 // The codes are exact: w * (1/Delta) is rounded unless it lands within 2^-18
 // of a half-integer (or 1/Delta is not finite), then the IEEE quotient is used.
 #pragma once
@@ -30,9 +33,10 @@
 
 namespace qat4 {
 
-constexpr int kRfTile = 64;          // refine_v_kernel output tile (rows x columns)
+constexpr int kRfTileR = 128;        // refine_v_kernel output tile: rows
+constexpr int kRfTileC = 64;         //                              columns
 constexpr int kRfK = 16;             // its reduction chunk
-constexpr int kRfWarps = 8;          // rows (warps) per sweep CTA
+constexpr int kRfWarps = 8;          // rows (warps) per sweep CTA, walking the groups in lockstep
 constexpr int kRfPacked = 528;       // 32 * 33 / 2 entries of a folded 32x32 block
 
 // Exact code of w at step dk with rc = 1/dk (see the file comment).
@@ -67,59 +71,99 @@ refine_err_kernel(const float* __restrict__ W, int64_t ngroups, const float* __r
     }
 }
 
-// V[r, :] = E[r, :] H (H symmetric), binary64 accumulation of exact products; 64 x 64 tiles.
-__global__ void __launch_bounds__(256)
+// V[r, :] = E[r, :] H (H symmetric), binary64: one accumulator per output, k ascending.  A
+// 256-thread CTA computes a 128 x 64 tile, each thread 8 rows x 4 columns; 16-deep chunks of E
+// (stored transposed, rows padded to 130 doubles so that the transposing stores spread over the
+// banks and every thread's 8 rows are two aligned 16-byte pairs) and of H (converted to binary64
+// once) go through shared memory, the next chunk's global loads held in registers meanwhile.
+__global__ void __launch_bounds__(256, 2)
 refine_v_kernel(const double* __restrict__ E, int R, int C, const float* __restrict__ H, int64_t ldh,
                 double* __restrict__ V) {
-    __shared__ double se[kRfTile][kRfK + 1];
-    __shared__ double sh[kRfK][kRfTile + 1];
-    const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    const int r0 = blockIdx.y * kRfTile, c0 = blockIdx.x * kRfTile;
-    double acc[4][4];
+    constexpr int kEPad = kRfTileR + 2;
+    __shared__ __align__(16) double se[kRfK][kEPad];
+    __shared__ __align__(16) double sh[kRfK][kRfTileC];
+    const int tid = threadIdx.x;
+    const int tx = tid & 15, ty = tid >> 4;
+    const int r0 = blockIdx.y * kRfTileR, c0 = blockIdx.x * kRfTileC;
+    double acc[8][4];
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
+    for (int a = 0; a < 8; ++a)
 #pragma unroll
         for (int b = 0; b < 4; ++b) acc[a][b] = 0.0;
+    // this thread's share of a chunk: E elements x = tid + 256 i (row x / 16, k x % 16: a row's 16
+    // values are 128 contiguous bytes), H elements y = tid + 256 i (k y / 64, column y % 64)
+    double pe[8];
+    float ph[4];
+    auto load = [&](int k0) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int x = tid + 256 * i, r = r0 + (x >> 4);
+            pe[i] = r < R ? E[static_cast<int64_t>(r) * C + k0 + (x & 15)] : 0.0;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int y = tid + 256 * i, c = c0 + (y & 63);
+            ph[i] = c < C ? H[static_cast<int64_t>(k0 + (y >> 6)) * ldh + c] : 0.0f;
+        }
+    };
+    auto stash = [&]() {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int x = tid + 256 * i;
+            se[x & 15][x >> 4] = pe[i];
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int y = tid + 256 * i;
+            sh[y >> 6][y & 63] = static_cast<double>(ph[i]);
+        }
+    };
+    load(0);
+    stash();
+    __syncthreads();
     for (int k0 = 0; k0 < C; k0 += kRfK) {
-        for (int x = threadIdx.x; x < kRfTile * kRfK; x += 256) {
-            const int rr = x / kRfK, kk = x % kRfK;
-            const int r = r0 + rr, k = k0 + kk;
-            se[rr][kk] = (r < R && k < C) ? E[static_cast<int64_t>(r) * C + k] : 0.0;
-        }
-        for (int x = threadIdx.x; x < kRfK * kRfTile; x += 256) {
-            const int kk = x / kRfTile, cc = x % kRfTile;
-            const int k = k0 + kk, c = c0 + cc;
-            sh[kk][cc] = (k < C && c < C) ? static_cast<double>(H[static_cast<int64_t>(k) * ldh + c]) : 0.0;
-        }
-        __syncthreads();
-#pragma unroll 4
+        const bool more = k0 + kRfK < C;
+        if (more) load(k0 + kRfK);
+#pragma unroll
         for (int kk = 0; kk < kRfK; ++kk) {
-            double ea[4], hb[4];
+            double ea[8], hb[4];
+            const double2* e2 = reinterpret_cast<const double2*>(&se[kk][ty * 8]);
+            const double2* h2 = reinterpret_cast<const double2*>(&sh[kk][tx * 4]);
 #pragma unroll
-            for (int a = 0; a < 4; ++a) ea[a] = se[ty * 4 + a][kk];
+            for (int q = 0; q < 4; ++q) {
+                const double2 t = e2[q];
+                ea[2 * q] = t.x;
+                ea[2 * q + 1] = t.y;
+            }
 #pragma unroll
-            for (int b = 0; b < 4; ++b) hb[b] = sh[kk][tx * 4 + b];
+            for (int q = 0; q < 2; ++q) {
+                const double2 t = h2[q];
+                hb[2 * q] = t.x;
+                hb[2 * q + 1] = t.y;
+            }
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < 8; ++a)
 #pragma unroll
                 for (int b = 0; b < 4; ++b) acc[a][b] = fma(ea[a], hb[b], acc[a][b]);
         }
         __syncthreads();
+        if (more) {
+            stash();
+            __syncthreads();
+        }
     }
 #pragma unroll
-    for (int a = 0; a < 4; ++a) {
-        const int r = r0 + ty * 4 + a;
-        if (r >= R) continue;
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const int c = c0 + tx * 4 + b;
-            if (c < C) V[static_cast<int64_t>(r) * C + c] = acc[a][b];
-        }
+    for (int a = 0; a < 8; ++a) {
+        const int r = r0 + ty * 8 + a;
+        const int c = c0 + tx * 4;
+        if (r >= R || c >= C) continue;                  // C % 32 == 0: a thread's 4 columns are all in or all out
+        double2* dst = reinterpret_cast<double2*>(V + static_cast<int64_t>(r) * C + c);
+        dst[0] = make_double2(acc[a][0], acc[a][1]);
+        dst[1] = make_double2(acc[a][2], acc[a][3]);
     }
 }
 
-struct RefineWarpSmem {
-    double hp[kRfPacked];    // H_gg folded: H_ii, then 2 H_ij for j > i, row by row
+struct RefineRowSmem {
     double u[32];            // u_g = v_g - H_gg e_g
     double delta[32];        // e'_g - e_g of a move
     float w[32];             // the group's weights
@@ -128,105 +172,127 @@ struct RefineWarpSmem {
 // Row i of a folded 32x32 block starts at i*32 - i*(i-1)/2 and holds columns i..31.
 __host__ __device__ constexpr int refine_tri(int i) { return i * 32 - i * (i - 1) / 2; }
 
+// The rows of a CTA (one warp each) walk the groups in lockstep, so that each group's block of H
+// is staged once per CTA and each group's 32 rows of H are read once per CTA for all of the
+// CTA's rows that move: (1) the CTA stages H_gg, full (binary32) and folded (binary64); (2) every
+// warp takes its row's decision; (3) the CTA adds H[c0.., :]^T (e'_g - e_g) into v of every row
+// that moved.  Each row's arithmetic is the same sequence as one warp alone would run.
 __global__ void __launch_bounds__(32 * kRfWarps)
 refine_sweep_kernel(const float* __restrict__ W, int R, int C, const float* __restrict__ H, int64_t ldh,
                     const float* __restrict__ alpha, int K, int sweeps, int32_t* __restrict__ idx,
                     float* __restrict__ delta_out, double* __restrict__ obj_out, double* __restrict__ V) {
-    __shared__ RefineWarpSmem sm[kRfWarps];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int r = blockIdx.x * kRfWarps + warp;
-    if (r >= R) return;                          // no block-wide synchronisation below
-    RefineWarpSmem& s = sm[warp];
+    __shared__ double hp[kRfPacked];         // H_gg folded: H_ii, then 2 H_ij for j > i, row by row
+    __shared__ float hf[32][33];             // H_gg as it is (row i: column j)
+    __shared__ RefineRowSmem rs[kRfWarps];
+    __shared__ unsigned moved;               // bit m: row m of the CTA moved at this group
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int r0 = blockIdx.x * kRfWarps;
+    const int r = r0 + warp;
+    const bool live = r < R;                 // every thread takes part in the CTA barriers
+    RefineRowSmem& s = rs[warp];
     const int G = C >> 5;
-    const float* wrow = W + static_cast<int64_t>(r) * C;
-    double* v = V + static_cast<int64_t>(r) * C;
-    int32_t* irow = idx + static_cast<int64_t>(r) * G;
+    const float* wrow = W + static_cast<int64_t>(live ? r : 0) * C;
+    double* v = V + static_cast<int64_t>(live ? r : 0) * C;
+    int32_t* irow = idx + static_cast<int64_t>(live ? r : 0) * G;
 
     for (int sw = 0; sw < sweeps; ++sw) {
         for (int g = 0; g < G; ++g) {
             const int c0 = g * 32;
-            const float wi = wrow[c0 + lane];
-            const float base = refine_base(wi);
-            s.w[lane] = wi;
-            // lane i: row i of H_gg, folded into the upper triangle
-            const float* hrow = H + static_cast<int64_t>(c0 + lane) * ldh + c0;
-            float hr[32];
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                const float4 t = *reinterpret_cast<const float4*>(hrow + j);
-                hr[j] = t.x; hr[j + 1] = t.y; hr[j + 2] = t.z; hr[j + 3] = t.w;
+            // (1) H_gg into shared memory
+            for (int x = tid; x < 32 * 32; x += 32 * kRfWarps) {
+                const int i = x >> 5, j = x & 31;
+                const float h = H[static_cast<int64_t>(c0 + i) * ldh + c0 + j];
+                hf[i][j] = h;
+                if (j >= i) hp[refine_tri(i) + j - i] = (j == i ? 1.0 : 2.0) * static_cast<double>(h);
             }
-            const int cur = min(max(irow[g], 0), K - 1);
-            const float dcur = __ldg(alpha + cur) * base;
-            const float qcur = code_of(scaled_exact(wi, dcur));
-            const double ecur = static_cast<double>(wi) - static_cast<double>(dcur * qcur);
-            // u_i = v_i - sum_j H_ij e_j (e_j from lane j)
-            double hu = 0.0;
-#pragma unroll
-            for (int j = 0; j < 32; ++j) hu = fma(static_cast<double>(hr[j]), __shfl_sync(0xffffffffu, ecur, j), hu);
-            s.u[lane] = v[c0 + lane] - hu;
-            {
-                const int t0 = refine_tri(lane);
+            if (tid == 0) moved = 0u;
+            __syncthreads();
+            // (2) this warp's row
+            if (live) {
+                const float wi = wrow[c0 + lane];
+                const float base = refine_base(wi);
+                s.w[lane] = wi;
+                const int cur = min(max(irow[g], 0), K - 1);
+                const float dcur = __ldg(alpha + cur) * base;
+                const float qcur = code_of(scaled_exact(wi, dcur));
+                const double ecur = static_cast<double>(wi) - static_cast<double>(dcur * qcur);
+                // u_i = v_i - sum_j H_ij e_j (e_j from lane j)
+                double hu = 0.0;
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
-                    if (j >= lane) s.hp[t0 + j - lane] = (j == lane ? 1.0 : 2.0) * static_cast<double>(hr[j]);
-            }
-            __syncwarp();
-            // candidates k = lane, lane + 32, ...: e' H_gg e'^T + 2 e'.u
-            double best = 0.0;
-            int best_k = -1;
-            for (int k = lane; k < K; k += 32) {
-                const float dk = __ldg(alpha + k) * base;
-                const float rc = __frcp_rn(dk);
-                const bool rc_ok = fabsf(rc) <= 3.4028234663852886e38f;
-                double e[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float wv = s.w[i];
-                    e[i] = static_cast<double>(wv) - static_cast<double>(dk * refine_code(wv, dk, rc, rc_ok));
-                }
-                double Ek = 0.0;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    double row = 2.0 * s.u[i];
-#pragma unroll
-                    for (int j = i; j < 32; ++j) row = fma(s.hp[refine_tri(i) + j - i], e[j], row);
-                    Ek = fma(e[i], row, Ek);
-                }
-                if (best_k < 0 || Ek < best) {
-                    best = Ek;
-                    best_k = k;
-                }
-            }
-            // warp argmin, ties to the smallest k (lanes without a candidate carry +inf)
-            if (best_k < 0) best = __longlong_as_double(0x7FF0000000000000ll);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const double ob = __shfl_xor_sync(0xffffffffu, best, o);
-                const int ok = __shfl_xor_sync(0xffffffffu, best_k, o);
-                if (ob < best || (ob == best && ok >= 0 && (best_k < 0 || ok < best_k))) {
-                    best = ob;
-                    best_k = ok;
-                }
-            }
-            if (best_k != cur) {
-                const float dnew = __ldg(alpha + best_k) * base;
-                const float qnew = code_of(scaled_exact(wi, dnew));
-                s.delta[lane] = (static_cast<double>(wi) - static_cast<double>(dnew * qnew)) - ecur;
+                    hu = fma(static_cast<double>(hf[lane][j]), __shfl_sync(0xffffffffu, ecur, j), hu);
+                s.u[lane] = v[c0 + lane] - hu;
                 __syncwarp();
-                // v_j += sum_i H[c0 + i][j] delta_i (H symmetric), lanes along j
-                for (int j = lane; j < C; j += 32) {
-                    double a = 0.0;
-#pragma unroll 8
-                    for (int i = 0; i < 32; ++i)
-                        a = fma(static_cast<double>(__ldg(H + static_cast<int64_t>(c0 + i) * ldh + j)), s.delta[i], a);
-                    v[j] += a;
+                // candidates k = lane, lane + 32, ...: e' H_gg e'^T + 2 e'.u
+                double best = 0.0;
+                int best_k = -1;
+                for (int k = lane; k < K; k += 32) {
+                    const float dk = __ldg(alpha + k) * base;
+                    const float rc = __frcp_rn(dk);
+                    const bool rc_ok = fabsf(rc) <= 3.4028234663852886e38f;
+                    double e[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const float wv = s.w[i];
+                        e[i] = static_cast<double>(wv) - static_cast<double>(dk * refine_code(wv, dk, rc, rc_ok));
+                    }
+                    double Ek = 0.0;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        double row = 2.0 * s.u[i];
+#pragma unroll
+                        for (int j = i; j < 32; ++j) row = fma(hp[refine_tri(i) + j - i], e[j], row);
+                        Ek = fma(e[i], row, Ek);
+                    }
+                    if (best_k < 0 || Ek < best) {
+                        best = Ek;
+                        best_k = k;
+                    }
                 }
-                if (lane == 0) irow[g] = best_k;
+                // warp argmin, ties to the smallest k (lanes without a candidate carry +inf)
+                if (best_k < 0) best = __longlong_as_double(0x7FF0000000000000ll);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+                    const int ok = __shfl_xor_sync(0xffffffffu, best_k, o);
+                    if (ob < best || (ob == best && ok >= 0 && (best_k < 0 || ok < best_k))) {
+                        best = ob;
+                        best_k = ok;
+                    }
+                }
+                if (best_k != cur) {
+                    const float dnew = __ldg(alpha + best_k) * base;
+                    const float qnew = code_of(scaled_exact(wi, dnew));
+                    s.delta[lane] = (static_cast<double>(wi) - static_cast<double>(dnew * qnew)) - ecur;
+                    if (lane == 0) {
+                        irow[g] = best_k;
+                        atomicOr(&moved, 1u << warp);
+                    }
+                }
             }
-            __syncwarp();
+            __syncthreads();
+            // (3) v_j += sum_i H[c0 + i][j] delta_i (H symmetric) for every row that moved; threads
+            // along j, so each of the group's 32 rows of H is read once for the whole CTA
+            const unsigned mm = moved;
+            if (mm != 0u) {
+                for (int j = tid; j < C; j += 32 * kRfWarps) {
+                    float hc[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) hc[i] = __ldg(H + static_cast<int64_t>(c0 + i) * ldh + j);
+                    for (unsigned left = mm; left != 0u; left &= left - 1u) {
+                        const int m = __ffs(left) - 1;
+                        double a = 0.0;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) a = fma(static_cast<double>(hc[i]), rs[m].delta[i], a);
+                        V[static_cast<int64_t>(r0 + m) * C + j] += a;
+                    }
+                }
+            }
+            __syncthreads();
         }
     }
+    if (!live) return;
     // outputs: Delta of every group and the final objective e . v
     double obj = 0.0;
     for (int g = 0; g < G; ++g) {
