@@ -15,7 +15,7 @@
 //   refine_err_kernel   e = w - fl(Delta q) for the starting indices, binary64
 //                       (exact: difference of two binary32 values);
 //   refine_v_kernel     V = E H, a tiled binary64 product (H read once per
-//                       64-row tile), into the caller's workspace;
+//                       128-row tile of E), into the caller's workspace;
 //   refine_sweep_kernel one warp per row, the CTA's rows walking the groups in
 //                       lockstep: u_g from v and the group's block of H (staged
 //                       once per CTA); every candidate's
