@@ -149,3 +149,32 @@ def test_lsq_host_validation():
     assert f(A, A, A, 5, 3000, 1024, s, A, A, A, B, ws, None, None) == 4             # dtype
     assert f(A, A, A, 1, 3000, 1024, s, A, A, A, B, ws - 1, None, None) == 5         # small workspace
     assert f(A, A, A, 1, 3000, 1024, s, A, A, A, ct.c_void_p(0x20010), ws, None, None) == 3  # alignment
+
+
+def _plan_workspace(n, C):
+    """The split of the calibration rows as the Hessian's planner states it: T upper 256x256 tiles
+    on 74 SM pairs; the tiles of the last (or only) wave are cut into min(74 // r, ceil(n/128) // 16)
+    parts when that is at least 2, and each cut tile keeps one 256x256 float32 partial per part."""
+    nb = -(-C // 256)
+    T = nb * (nb + 1) // 2
+    r = T if T <= 74 else T % 74
+    s = min(74 // r if r else 1, -(-n // 128) // 16)
+    return 0 if (s < 2 or r == 0) else r * s * 256 * 256 * 4
+
+
+@pytest.mark.parametrize("n,C", [(262144, 2048), (40000, 3072), (262144, 8192), (131072, 14336),
+                                 (131072, 4096), (1000, 2048), (4096, 512), (16, 32), (262144, 65536)])
+def test_hessian_workspace_follows_the_split_plan(n, C):
+    """Host-side plan, no GPU: the workspace the library asks for is the plan's partial tiles."""
+    import int4_group_wise_b200 as q4
+    assert q4.hessian_workspace_bytes(n, C) == _plan_workspace(n, C)
+
+
+def test_hessian_workspace_examples():
+    """The 1B-class up-projection splits all 36 tiles in two (18.9 MB of partials); 78 tiles put the
+    4 of the second wave in 18 parts; 528 tiles leave 10 for the last wave, cut in 7."""
+    import int4_group_wise_b200 as q4
+    assert q4.hessian_workspace_bytes(262144, 2048) == 36 * 2 * 262144
+    assert q4.hessian_workspace_bytes(40000, 3072) == 4 * 18 * 262144
+    assert q4.hessian_workspace_bytes(262144, 8192) == 10 * 7 * 262144
+    assert q4.hessian_workspace_bytes(0, 2048) == 0 and q4.hessian_workspace_bytes(100, 48) == 0
